@@ -1,0 +1,214 @@
+/*
+ * moe_mxfp4.h -- C ABI of the MXFP4 Mixture-of-Experts layer library
+ * (libmoe_mxfp4.so, built for NVIDIA B200 / sm_100a).
+ *
+ * The operation is the MoE MLP block of a GPT-OSS-style decoder:
+ *   - token-choice routing, each token picking its top-k experts, with the
+ *     softmax taken over the k selected logits only ("softmax-after-topk")
+ *     ["Welcome GPT OSS, the new open-source model family from OpenAI"
+ *      (summary), section 4 "MoE, quantisation and context handling"];
+ *   - 4 active experts per token, 32 or 128 experts per layer, independent
+ *     experts with no shared expert [aitrends.kr talk summary, chapters
+ *     "Architecture details: MoE and attention" and "Q&A"];
+ *   - SwiGLU experts whose weights are MXFP4: E2M1 4-bit elements (1 sign,
+ *     2 exponent, 1 mantissa bit) with one shared scale per block of 32
+ *     elements ["Tricks from OpenAI gpt-oss you can use with transformers"
+ *     (summary), section 6 "MXFP4 format and memory savings";
+ *     agentlenshq "Transformers ... GPT-OSS" (ja), section "What is MXFP4"];
+ *     the format is the OCP Microscaling (MX) one, so the shared scale is an
+ *     E8M0 power of two ["MXFP4-based MoE technical review", section 1];
+ *   - weights stay 4-bit in memory and are raised to bf16 only inside the
+ *     GEMM [aitrends.kr talk summary, chapter "Hardware optimisation"];
+ *     GEMM kernels must understand the 32-element blocks and their scales
+ *     ["Tricks from OpenAI gpt-oss ...", section 8].
+ *
+ * Notation: T tokens, E experts, k experts per token, D = d_model,
+ * F = d_ff, S = T*k routed slots; slot s = t*k + j, j = rank within the
+ * token's top-k (j = 0 is the highest logit).
+ *
+ * Data layouts (all row-major, all pointers are DEVICE pointers unless a
+ * function says otherwise; bf16 values travel as raw uint16_t bit patterns):
+ *   x          bf16  [T][D]
+ *   logits     fp32  [T][E]
+ *   w_gu       MXFP4 [E][2F][D]  rows [0,F) are the gate projection,
+ *                                rows [F,2F) the up projection; the 32-blocks
+ *                                run along D (the reduction axis).
+ *   w_dn       MXFP4 [E][D][F]   32-blocks run along F.
+ *   An MXFP4 matrix [R][K] is two arrays:
+ *     q  uint8 [R][K/2]   element 2i in the low nibble of byte i, element
+ *                         2i+1 in the high nibble; nibble = sign<<3 | e<<1 | m
+ *     s  uint8 [R][K/32]  E8M0 scale byte b, scale = 2^(b-127)
+ *   value = (-1)^sign * {0,0.5,1,1.5,2,3,4,6}[nibble & 7] * 2^(b-127).
+ *
+ * Conventions shared by every call:
+ *   - Ownership: the caller allocates and owns every buffer, including the
+ *     workspace; the library never allocates, never synchronises the device
+ *     and never falls back to another implementation.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed
+ *     as void*; NULL = the legacy default stream).
+ *   - Host-side validation (null pointers, shapes, alignment, workspace
+ *     size, device architecture) happens before anything is launched; on
+ *     failure the call returns the status and launches nothing.
+ *   - MOE_ERR_CUDA is returned when a kernel launch reports an error.
+ *   - Conditions only the device can see (non-finite quantiser input, a
+ *     bounded wait that gave up) are written to a device status word
+ *     (`d_status`, or the first 4 bytes of the workspace); the caller reads
+ *     it after synchronising.  Kernels never trap or assert.
+ *   - Calls on different streams with different workspaces are independent.
+ *   - Every device pointer must be 16-byte aligned.
+ */
+#ifndef MOE_MXFP4_H
+#define MOE_MXFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, misaligned pointer, bad enum   */
+  MOE_ERR_SHAPE = 2,       /* shape outside the supported range           */
+  MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
+  MOE_ERR_UNSUPPORTED = 4, /* current device is not compute capability 10.0 */
+  MOE_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed        */
+  MOE_ERR_NONFINITE = 6,   /* device status only: NaN/Inf quantiser input */
+  MOE_ERR_TIMEOUT = 7      /* device status only: a bounded wait gave up  */
+} moe_status;
+
+/* Shape of one MoE layer call.
+ * Supported: 1 <= T <= 1<<20, 1 <= E <= 256, 1 <= k <= min(E, 8),
+ * D and F multiples of 64 in [64, 16384], T*k < 2^31.                    */
+typedef struct {
+  int32_t T;
+  int32_t E;
+  int32_t k;
+  int32_t d_model;
+  int32_t d_ff;
+} moe_shape;
+
+typedef void* moe_stream; /* cudaStream_t */
+
+/* mxfp4_quantize -- bf16 -> MXFP4 block quantiser.
+ * Passage: E2M1 with a 32-element shared scale ("Tricks from OpenAI
+ * gpt-oss ...", section 6; agentlenshq (ja), "What is MXFP4"), OCP MX
+ * E8M0 scale ("MXFP4-based MoE technical review", section 1).
+ * Per 32-element block of each row: amax = max |x|; scale byte
+ * b = clamp(bexp(amax) - 2, 0, 254), where bexp is the 8-bit exponent field
+ * of amax (so b = floor(log2 amax) - 2 + 127 for normal amax, 0 for a zero
+ * or subnormal amax); each element is |x| / 2^(b-127) rounded to nearest,
+ * ties to even mantissa, onto {0,0.5,1,1.5,2,3,4,6}, saturating at 6; the
+ * sign bit is the sign of x (so -0 and small negatives give code 8).
+ *   w_bf16   in   [rows][K] bf16
+ *   rows     in   >= 0 (0 is a no-op), rows*K < 2^40
+ *   K        in   multiple of 32, >= 32
+ *   q_packed out  [rows][K/2]
+ *   scales   out  [rows][K/32]
+ *   d_status out  nullable; if a block holds NaN or Inf the kernel stores
+ *                 MOE_ERR_NONFINITE there (that block's bytes are
+ *                 unspecified); it never writes MOE_OK, so clear it first.
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA.                                                          */
+moe_status mxfp4_quantize(const uint16_t* w_bf16, int64_t rows, int64_t K,
+                          uint8_t* q_packed, uint8_t* scales,
+                          int32_t* d_status, moe_stream stream);
+
+/* moe_route -- token-choice top-k with softmax over the chosen k.
+ * Passage: "Welcome GPT OSS ..." (summary), section 4 (token-choice MoE,
+ * softmax-after-topk); aitrends.kr talk summary (4 active experts).
+ * Per token t: the k experts with the largest logits, ordered by
+ * (logit descending, expert index ascending) -- equal logits, including
+ * -0 and +0, go to the lower index; topk_w[t][j] = softmax over those k
+ * logits, computed in fp32.
+ *   logits   in   [T][E] fp32, finite
+ *   topk_idx out  [T][k] int32
+ *   topk_w   out  [T][k] fp32
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA.                                                          */
+moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
+                     int32_t* topk_idx, float* topk_w, moe_stream stream);
+
+/* moe_permute -- group the T*k routed slots by expert.
+ * Passage: "MXFP4-based MoE technical review", section 4 (routing and its
+ * parallelisation as the core difficulty of sparse experts).
+ *   topk_idx    in   [T][k] int32, every entry in [0, E)
+ *   x           in   [T][D] bf16
+ *   counts      out  [E]   slots routed to each expert
+ *   offsets     out  [E+1] exclusive prefix sum of counts (offsets[E] = S)
+ *   sorted_slot out  [S]   slots grouped by expert (experts ascending),
+ *                          ascending slot order inside each expert
+ *   slot_pos    out  [S]   inverse: sorted_slot[slot_pos[s]] == s
+ *   x_perm      out  [S][D] bf16, x_perm[p] = x[sorted_slot[p] / k]
+ *   ws          in   device workspace of moe_workspace_size(shape, 0) bytes
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_WORKSPACE,
+ * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.                                     */
+moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x,
+                       moe_shape shape, int32_t* counts, int32_t* offsets,
+                       int32_t* sorted_slot, int32_t* slot_pos,
+                       uint16_t* x_perm, void* ws, size_t ws_bytes,
+                       moe_stream stream);
+
+/* moe_expert_mlp -- grouped SwiGLU expert MLP on MXFP4 weights.
+ * Passage: SwiGLU experts ("Welcome GPT OSS ...", section 4); MXFP4-aware
+ * GEMMs ("Tricks from OpenAI gpt-oss ...", section 8); weights raised to
+ * bf16 only for compute (aitrends.kr, "Hardware optimisation").
+ * For every expert e and every permuted row r in [offsets[e], offsets[e+1]):
+ *   g = x_perm[r] . Wg_e^T, u = x_perm[r] . Wu_e^T   (fp32 accumulation of
+ *                                                    exact bf16 products)
+ *   h[r] = bf16_rne(silu(g) * u),   silu(g) = g / (1 + exp(-g))
+ *   y_perm[r] = bf16_rne(h[r] . Wd_e^T)
+ *   x_perm  in   [S][D] bf16
+ *   offsets in   [E+1] as produced by moe_permute
+ *   wgu_q/s in   MXFP4 [E][2F][D]; wdn_q/s in MXFP4 [E][D][F]
+ *   h       out  [S][F] bf16 (caller-owned intermediate)
+ *   y_perm  out  [S][D] bf16
+ *   ws      in   device workspace of moe_workspace_size(shape, 1) bytes
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_WORKSPACE,
+ * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA; device status MOE_ERR_TIMEOUT.      */
+moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets,
+                          moe_shape shape, const uint8_t* wgu_q,
+                          const uint8_t* wgu_s, const uint8_t* wdn_q,
+                          const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm,
+                          void* ws, size_t ws_bytes, moe_stream stream);
+
+/* moe_combine -- routing-weighted, deterministic gather-sum.
+ * Passage: "Welcome GPT OSS ..." (summary), section 4 (the softmax weights
+ * of the chosen experts mix their outputs).
+ * out[t][d] = bf16_rne( sum_{j=0..k-1, ascending} topk_w[t][j] *
+ *                       y_perm[slot_pos[t*k+j]][d] ), summed in fp32.
+ *   y_perm   in  [S][D] bf16; slot_pos in [S]; topk_w in [T][k] fp32
+ *   out      out [T][D] bf16
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA.                                                          */
+moe_status moe_combine(const uint16_t* y_perm, const int32_t* slot_pos,
+                       const float* topk_w, moe_shape shape, uint16_t* out,
+                       moe_stream stream);
+
+/* moe_layer_forward -- the whole layer: moe_route -> moe_permute ->
+ * moe_expert_mlp -> moe_combine, enqueued on one stream, all intermediates
+ * in the caller's workspace (moe_workspace_size(shape, 2) bytes).
+ *   x in [T][D] bf16; logits in [T][E] fp32; weights as moe_expert_mlp;
+ *   out out [T][D] bf16.  The first 4 bytes of ws are the device status
+ *   word; the call resets it to MOE_OK before its first kernel.
+ * Errors: the union of the four calls.                                   */
+moe_status moe_layer_forward(const uint16_t* x, const float* logits,
+                             moe_shape shape, const uint8_t* wgu_q,
+                             const uint8_t* wgu_s, const uint8_t* wdn_q,
+                             const uint8_t* wdn_s, uint16_t* out, void* ws,
+                             size_t ws_bytes, moe_stream stream);
+
+/* moe_workspace_size -- bytes of device workspace a call needs.
+ * which: 0 = moe_permute, 1 = moe_expert_mlp, 2 = moe_layer_forward.
+ * Returns 0 for an unsupported shape or an unknown `which`.  Host only.  */
+size_t moe_workspace_size(moe_shape shape, int which);
+
+/* moe_status_string -- static, human-readable name of a status. */
+const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_MXFP4_H */
