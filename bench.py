@@ -1,0 +1,422 @@
+"""Benchmark of the MXFP4 MoE layer (one JSON line on stdout from rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one moe_layer_forward call (route -> permute -> grouped gate/up
+GEMM + SwiGLU -> grouped down GEMM -> combine) over one batch of seeded
+synthetic tokens with the workload's shapes; the MXFP4 weights are quantised
+once, before timing, by the library's mxfp4_quantize.  L2 is flushed (a
+256 MiB device write) before every timed step, outside the timed events.
+
+* value: tokens/s of the whole job (all ranks), inputs resident in HBM, from
+  CUDA events around each step on the launching stream, max over ranks.
+* e2e: the same metric through the same C-ABI call with host buffers: the
+  step's x and logits are copied from pinned host memory and the output is
+  copied back inside the timed region.
+* roofline: the grouped expert MLP (moe_expert_mlp: the two GEMM launches
+  that dominate the step), algorithmic bytes per call / its event time,
+  against the measured HBM copy bandwidth.
+* cpu_baseline: the fp64 CPU oracle, as it stands, on the host cores, over a
+  bounded sample of the same workload (rank 0, one GPU only).
+Under torchrun each rank runs its own replica of the workload on its own GPU
+(independent token batches, no collective on the data path): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as syn  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200; % of roofline (HBM GB/s decode, TC TFLOP/s prefill)"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "20b_decode"
+FLUSH_BYTES = 256 << 20
+# kernel launches of one moe_layer_forward call: route, permute (bookkeeping +
+# row gather), expert MLP (gate/up, down), combine
+LAUNCHES_PER_LAYER = 6
+# dram bytes (read + write) of one moe_expert_mlp call on the default workload,
+# from an ncu capture of the kernels whose source hashes to TRAFFIC_SRC_SHA;
+# reported only while the source is unchanged
+TRAFFIC_BYTES = None
+TRAFFIC_SRC_SHA = None
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def expert_bytes(wl) -> int:
+    D, F = wl.d_model, wl.d_ff
+    return 2 * F * D // 2 + 2 * F * D // 32 + D * F // 2 + D * F // 32
+
+
+def kernel_src_sha() -> str:
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "mxfp4_quantised_mixture_b200", "csrc", "expert_mlp.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- reference arm
+
+
+def cpu_oracle_sample(wl, n_tokens: int, weights=None):
+    """Time the fp64 oracle over the first n_tokens of the workload.
+    Returns (seconds, tokens, threads, weights)."""
+    import oracle
+
+    x = syn.activations(wl)
+    lg = syn.logits(wl)
+    tokens = list(range(min(n_tokens, wl.T)))
+    if weights is None:
+        idx, _ = oracle.route(lg[tokens], wl.k)
+        need = sorted(set(int(v) for v in idx.ravel()))
+        D, F, E = wl.d_model, wl.d_ff, wl.E
+        gq = np.zeros((E, 2 * F, D // 2), np.uint8)
+        gs = np.zeros((E, 2 * F, D // 32), np.uint8)
+        dq = np.zeros((E, D, F // 2), np.uint8)
+        ds = np.zeros((E, D, F // 32), np.uint8)
+        for e in need:
+            q, s = oracle.quantize_experts(syn.w_gate_up(wl, [e]))
+            gq[e], gs[e] = q[0], s[0]
+            q, s = oracle.quantize_experts(syn.w_down(wl, [e]))
+            dq[e], ds[e] = q[0], s[0]
+        weights = (gq, gs, dq, ds)
+    t0 = time.perf_counter()
+    if len(tokens) == wl.T:
+        oracle.layer_forward(x, lg, wl.k, *weights)
+    else:
+        oracle.layer_tokens(x, lg, wl.k, *weights, tokens)
+    dt = time.perf_counter() - t0
+    return dt, len(tokens), max(1, min(64, os.cpu_count() or 1)), weights
+
+
+def reference_sample_tokens(wl) -> int:
+    return min(wl.T, 4)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = syn.WORKLOADS[args.workload]
+    n = reference_sample_tokens(wl)
+    weights = None
+    for _ in range(args.warmup):
+        _, _, _, weights = cpu_oracle_sample(wl, n, weights)
+    total = 0.0
+    threads = 1
+    for _ in range(args.steps):
+        dt, tok, threads, weights = cpu_oracle_sample(wl, n, weights)
+        total += dt
+    value = args.steps * n / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n} of {wl.T} tokens per step, first tokens of the batch, "
+                                   "weights of the experts they route to quantised before timing"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(wl):
+    return {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E,
+            "k": wl.k, "seed": wl.seed, "weights": "MXFP4 (E2M1 + E8M0 per 32), bf16 activations",
+            "l2": "flushed before every timed step (256 MiB device write, outside the events)",
+            "parallelism": "replica per GPU"}
+
+
+# -------------------------------------------------------------------- ours
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_quantised_mixture_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = syn.WORKLOADS[args.workload]
+    D, F, E, T, k = wl.d_model, wl.d_ff, wl.E, wl.T, wl.k
+    S = T * k
+    shape = moe.make_shape(T, E, k, D, F)
+
+    # ---- inputs (seeded, synthetic) and weights quantised by the library
+    x_np = syn.activations(wl)
+    lg_np = syn.logits(wl)
+    x = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    logits = torch.from_numpy(lg_np).to(dev)
+    wgu_q = torch.empty((E, 2 * F, D // 2), dtype=torch.uint8, device=dev)
+    wgu_s = torch.empty((E, 2 * F, D // 32), dtype=torch.uint8, device=dev)
+    wdn_q = torch.empty((E, D, F // 2), dtype=torch.uint8, device=dev)
+    wdn_s = torch.empty((E, D, F // 32), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    chunk = max(1, min(E, (1 << 28) // (2 * F * D)))
+    for e0 in range(0, E, chunk):
+        ex = list(range(e0, min(E, e0 + chunk)))
+        gu = torch.from_numpy(syn.w_gate_up(wl, ex).view(np.int16)).to(dev).view(torch.bfloat16)
+        dn = torch.from_numpy(syn.w_down(wl, ex).view(np.int16)).to(dev).view(torch.bfloat16)
+        moe.mxfp4_quantize(gu, wgu_q[e0:e0 + len(ex)], wgu_s[e0:e0 + len(ex)], status)
+        moe.mxfp4_quantize(dn, wdn_q[e0:e0 + len(ex)], wdn_s[e0:e0 + len(ex)], status)
+        del gu, dn
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError("quantiser reported non-finite weights")
+
+    out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    ws = moe.alloc_workspace(shape, moe.WS_LAYER, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def layer():
+        moe.moe_layer_forward(x, logits, shape, wgu_q, wgu_s, wdn_q, wdn_s, out, ws, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        layer()
+    torch.cuda.synchronize()
+    if int(ws[:4].view(torch.int32).item()) != 0:
+        raise RuntimeError("layer reported device status %d" % int(ws[:4].view(torch.int32).item()))
+
+    # ---- timed region: K steps, events around each step, L2 flushed between
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        layer()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    # ---- roofline of the grouped expert MLP: the same step through the
+    #      individual calls, with events around moe_expert_mlp
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    tw = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    ss = torch.empty(S, dtype=torch.int32, device=dev)
+    sp = torch.empty(S, dtype=torch.int32, device=dev)
+    xp = torch.empty((S, D), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((S, F), dtype=torch.bfloat16, device=dev)
+    yp = torch.empty((S, D), dtype=torch.bfloat16, device=dev)
+    ws_mlp = moe.alloc_workspace(shape, moe.WS_EXPERT_MLP, dev)
+    m_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    m_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps + 2):
+        flush.fill_(i & 0xFF)
+        moe.moe_route(logits, k, idx, tw, stream)
+        moe.moe_permute(idx, x, shape, counts, offsets, ss, sp, xp, None, stream)
+        if i >= 2:
+            m_starts[i - 2].record(stream)
+        moe.moe_expert_mlp(xp, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, yp, ws_mlp, stream)
+        if i >= 2:
+            m_ends[i - 2].record(stream)
+        moe.moe_combine(yp, sp, tw, shape, out, stream)
+    torch.cuda.synchronize()
+    mlp_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(m_starts, m_ends))
+    touched = int((counts > 0).sum().item())
+    mlp_bytes = touched * expert_bytes(wl) + 2 * S * D * 2
+    hbm, tc_burst, tc_sust, peak_kind = peaks()
+    achieved = mlp_bytes / (mlp_ms / 1e3) / 1e9
+    traffic = TRAFFIC_BYTES if (TRAFFIC_BYTES is not None and TRAFFIC_SRC_SHA == kernel_src_sha()) else None
+    layer_bytes = touched * expert_bytes(wl) + T * D * 2 + T * E * 4 + T * D * 2
+    layer_flops = 6.0 * S * D * F
+    t_roof_meas = max(layer_bytes / (hbm * 1e9), layer_flops / (tc_sust * 1e12))
+    t_roof_spec = max(layer_bytes / 8e12, layer_flops / 2.25e15)
+
+    # ---- end to end through the C ABI with host buffers
+    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_host = torch.from_numpy(lg_np).pin_memory()
+    out_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e_starts[i].record(stream)
+        x.copy_(x_host, non_blocking=True)
+        logits.copy_(lg_host, non_blocking=True)
+        layer()
+        out_host.copy_(out, non_blocking=True)
+        e_ends[i].record(stream)
+        e_ends[i].synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": x_host.numel() * 2 + lg_host.numel() * 4,
+           "d2h_bytes_per_step": out_host.numel() * 2}
+
+    # ---- CPU baseline (rank 0, one GPU)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = wl.T if wl.T <= 128 else 16
+        dt, tok, threads, _ = cpu_oracle_sample(wl, n)
+        cpu = {"value": tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": (f"all {tok} tokens of the batch" if tok == wl.T else
+                          f"first {tok} of {wl.T} tokens") +
+                         "; weights quantised by the oracle before timing"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(wl),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic,
+                     "kernel": "moe_expert_mlp (grouped gate/up+SwiGLU and down GEMMs)",
+                     "algorithmic_bytes": mlp_bytes, "ms": mlp_ms, "peak_source": peak_kind},
+        "layer_roofline": {"bytes": layer_bytes, "flops": layer_flops,
+                           "frac_of_measured": t_roof_meas / (ms_per_step / 1e3),
+                           "frac_of_spec_8TBs_2.25PF": t_roof_spec / (ms_per_step / 1e3),
+                           "touched_experts": touched},
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+        "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
+        "wall_s_timed_region": wall, "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -91,6 +91,14 @@ typedef struct {
 
 typedef void* moe_stream; /* cudaStream_t */
 
+/* exported symbols keep default visibility even when the library is built
+ * with -fvisibility=hidden */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
 /* mxfp4_quantize -- bf16 -> MXFP4 block quantiser.
  * Passage: E2M1 with a 32-element shared scale ("Tricks from OpenAI
  * gpt-oss ...", section 6; agentlenshq (ja), "What is MXFP4"), OCP MX
@@ -111,7 +119,7 @@ typedef void* moe_stream; /* cudaStream_t */
  *                 unspecified); it never writes MOE_OK, so clear it first.
  * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED,
  * MOE_ERR_CUDA.                                                          */
-moe_status mxfp4_quantize(const uint16_t* w_bf16, int64_t rows, int64_t K,
+MOE_API moe_status mxfp4_quantize(const uint16_t* w_bf16, int64_t rows, int64_t K,
                           uint8_t* q_packed, uint8_t* scales,
                           int32_t* d_status, moe_stream stream);
 
@@ -127,7 +135,7 @@ moe_status mxfp4_quantize(const uint16_t* w_bf16, int64_t rows, int64_t K,
  *   topk_w   out  [T][k] fp32
  * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED,
  * MOE_ERR_CUDA.                                                          */
-moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
+MOE_API moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
                      int32_t* topk_idx, float* topk_w, moe_stream stream);
 
 /* moe_permute -- group the T*k routed slots by expert.
@@ -144,7 +152,7 @@ moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
  *   ws          in   device workspace of moe_workspace_size(shape, 0) bytes
  * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_WORKSPACE,
  * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.                                     */
-moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x,
+MOE_API moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x,
                        moe_shape shape, int32_t* counts, int32_t* offsets,
                        int32_t* sorted_slot, int32_t* slot_pos,
                        uint16_t* x_perm, void* ws, size_t ws_bytes,
@@ -167,7 +175,7 @@ moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x,
  *   ws      in   device workspace of moe_workspace_size(shape, 1) bytes
  * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_WORKSPACE,
  * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA; device status MOE_ERR_TIMEOUT.      */
-moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets,
+MOE_API moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets,
                           moe_shape shape, const uint8_t* wgu_q,
                           const uint8_t* wgu_s, const uint8_t* wdn_q,
                           const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm,
@@ -182,7 +190,7 @@ moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets,
  *   out      out [T][D] bf16
  * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED,
  * MOE_ERR_CUDA.                                                          */
-moe_status moe_combine(const uint16_t* y_perm, const int32_t* slot_pos,
+MOE_API moe_status moe_combine(const uint16_t* y_perm, const int32_t* slot_pos,
                        const float* topk_w, moe_shape shape, uint16_t* out,
                        moe_stream stream);
 
@@ -193,7 +201,7 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* slot_pos,
  *   out out [T][D] bf16.  The first 4 bytes of ws are the device status
  *   word; the call resets it to MOE_OK before its first kernel.
  * Errors: the union of the four calls.                                   */
-moe_status moe_layer_forward(const uint16_t* x, const float* logits,
+MOE_API moe_status moe_layer_forward(const uint16_t* x, const float* logits,
                              moe_shape shape, const uint8_t* wgu_q,
                              const uint8_t* wgu_s, const uint8_t* wdn_q,
                              const uint8_t* wdn_s, uint16_t* out, void* ws,
@@ -202,10 +210,10 @@ moe_status moe_layer_forward(const uint16_t* x, const float* logits,
 /* moe_workspace_size -- bytes of device workspace a call needs.
  * which: 0 = moe_permute, 1 = moe_expert_mlp, 2 = moe_layer_forward.
  * Returns 0 for an unsupported shape or an unknown `which`.  Host only.  */
-size_t moe_workspace_size(moe_shape shape, int which);
+MOE_API size_t moe_workspace_size(moe_shape shape, int which);
 
 /* moe_status_string -- static, human-readable name of a status. */
-const char* moe_status_string(moe_status status);
+MOE_API const char* moe_status_string(moe_status status);
 
 #ifdef __cplusplus
 }

@@ -51,6 +51,8 @@ def _L():
         lib.oracle_mxfp4_value.restype = dbl
         lib.oracle_mxfp4_quantize.argtypes = [vp, i64, i64, vp, vp]
         lib.oracle_mxfp4_quantize.restype = i64
+        lib.oracle_mxfp4_quantize_mt.argtypes = [vp, i64, i64, vp, vp, i32]
+        lib.oracle_mxfp4_quantize_mt.restype = i64
         lib.oracle_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp]
         lib.oracle_route.argtypes = [vp, i64, i32, i32, vp, vp]
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
@@ -102,7 +104,7 @@ def mxfp4_quantize(w_bf16: np.ndarray) -> tuple[np.ndarray, np.ndarray, int]:
     rows = w.size // K if K else 0
     q = np.empty(w.shape[:-1] + (K // 2,), dtype=np.uint8)
     s = np.empty(w.shape[:-1] + (K // 32,), dtype=np.uint8)
-    bad = _L().oracle_mxfp4_quantize(_p(w), rows, K, _p(q), _p(s))
+    bad = _L().oracle_mxfp4_quantize_mt(_p(w), rows, K, _p(q), _p(s), _threads())
     return q, s, int(bad)
 
 

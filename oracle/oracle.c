@@ -122,14 +122,12 @@ static uint8_t e2m1_magnitude_code(double v) {
   return 7;                 /* (5, inf) -> 6.0, saturating            */
 }
 
-/* bf16 [rows][K] -> codes [rows][K/2] + scale bytes [rows][K/32].
- * Returns the number of blocks holding a NaN or infinity (their bytes are
- * not meaningful). */
-int64_t oracle_mxfp4_quantize(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q,
-                              uint8_t* s) {
+/* rows [r0, r1) of the quantiser below */
+static int64_t quantize_rows(const uint16_t* w, int64_t r0, int64_t r1, int64_t K, uint8_t* q,
+                             uint8_t* s) {
   int64_t bad = 0;
   const int64_t nb = K / 32;
-  for (int64_t r = 0; r < rows; ++r) {
+  for (int64_t r = r0; r < r1; ++r) {
     for (int64_t b = 0; b < nb; ++b) {
       const uint16_t* blk = w + r * K + b * 32;
       int nonfinite = 0;
@@ -152,6 +150,53 @@ int64_t oracle_mxfp4_quantize(const uint16_t* w, int64_t rows, int64_t K, uint8_
     }
   }
   return bad;
+}
+
+typedef struct {
+  const uint16_t* w;
+  int64_t r0, r1, K;
+  uint8_t *q, *s;
+  int64_t bad;
+} quant_job;
+
+static void* quant_run(void* arg) {
+  quant_job* j = (quant_job*)arg;
+  j->bad = quantize_rows(j->w, j->r0, j->r1, j->K, j->q, j->s);
+  return NULL;
+}
+
+/* bf16 [rows][K] -> codes [rows][K/2] + scale bytes [rows][K/32], rows split
+ * over threads (each row is independent).  Returns the number of blocks
+ * holding a NaN or infinity (their bytes are not meaningful). */
+int64_t oracle_mxfp4_quantize_mt(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q,
+                                 uint8_t* s, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if (rows < 64) nthreads = 1;
+  pthread_t th[256];
+  quant_job jobs[256];
+  int created[256];
+  int64_t chunk = (rows + nthreads - 1) / nthreads;
+  int used = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    quant_job j = {w, t * chunk, (t + 1) * chunk < rows ? (t + 1) * chunk : rows, K, q, s, 0};
+    jobs[t] = j;
+    if (jobs[t].r0 >= jobs[t].r1) break;
+    created[t] = pthread_create(&th[t], NULL, quant_run, &jobs[t]) == 0;
+    if (!created[t]) quant_run(&jobs[t]);
+    used = t + 1;
+  }
+  int64_t bad = 0;
+  for (int t = 0; t < used; ++t) {
+    if (created[t]) pthread_join(th[t], NULL);
+    bad += jobs[t].bad;
+  }
+  return bad;
+}
+
+int64_t oracle_mxfp4_quantize(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q,
+                              uint8_t* s) {
+  return quantize_rows(w, 0, rows, K, q, s);
 }
 
 /* codes + scales [rows][K] -> double values */

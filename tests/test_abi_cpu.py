@@ -1,0 +1,95 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+that include/*.h declares, and rejects bad arguments on the host before it
+touches the device (no compute calls here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import mxfp4_quantised_mixture_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names += re.findall(r"^MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_header_declares_the_six_calls_and_helpers():
+    names = declared_functions()
+    for n in ["mxfp4_quantize", "moe_route", "moe_permute", "moe_expert_mlp", "moe_combine",
+              "moe_layer_forward", "moe_workspace_size", "moe_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_library_needs_no_cuda_shared_library():
+    # cudart is linked statically and the driver is reached at run time, so
+    # the library loads where no GPU driver is installed
+    with open("/proc/self/maps") as f:
+        maps = f.read()
+    assert moe.LIB_PATH in maps
+
+
+def test_status_strings():
+    assert moe.moe_status_string(0) == "MOE_OK"
+    assert moe.moe_status_string(3) == "MOE_ERR_WORKSPACE"
+    assert moe.moe_status_string(7) == "MOE_ERR_TIMEOUT"
+    assert moe.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_workspace_size_is_host_only_and_monotone():
+    small = moe.make_shape(64, 32, 4, 2880, 2880)
+    big = moe.make_shape(8192, 32, 4, 2880, 2880)
+    a = moe.moe_workspace_size(small, moe.WS_LAYER)
+    b = moe.moe_workspace_size(big, moe.WS_LAYER)
+    assert 0 < a < b
+    S = 8192 * 4
+    # the layer workspace holds at least x_perm, h and y_perm (bf16)
+    assert b >= S * 2880 * 2 * 3
+    assert moe.moe_workspace_size(small, 9) == 0
+    assert moe.moe_workspace_size(moe.make_shape(64, 300, 4, 2880, 2880), moe.WS_LAYER) == 0
+
+
+@pytest.mark.parametrize("shape", [
+    (64, 0, 4, 2880, 2880),      # E = 0
+    (64, 32, 9, 2880, 2880),     # k > 8
+    (64, 4, 5, 2880, 2880),      # k > E
+    (64, 32, 4, 2880, 2890),     # F not a multiple of 64
+    (64, 32, 4, 32, 2880),       # D too small
+    (-1, 32, 4, 2880, 2880),     # T < 0
+])
+def test_bad_shapes_rejected_before_the_device(shape):
+    sh = moe.make_shape(*shape)
+    st = moe.lib.moe_layer_forward(16, 16, sh, 16, 16, 16, 16, 16, 16, 1 << 30, None)
+    assert st == moe.MOE_ERR_SHAPE
+    st = moe.lib.moe_expert_mlp(16, 16, sh, 16, 16, 16, 16, 16, 16, 16, 1 << 30, None)
+    assert st == moe.MOE_ERR_SHAPE
+
+
+def test_bad_arguments_rejected_before_the_device():
+    L = moe.lib
+    assert L.mxfp4_quantize(16, 4, 48, 16, 16, None, None) == moe.MOE_ERR_SHAPE  # K % 32
+    assert L.mxfp4_quantize(None, 4, 64, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.mxfp4_quantize(24, 4, 64, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG  # misaligned
+    assert L.mxfp4_quantize(16, 0, 64, 16, 16, None, None) == moe.MOE_OK  # empty: no-op
+    assert L.moe_route(16, 4, 300, 4, 16, 16, None) == moe.MOE_ERR_SHAPE
+    assert L.moe_route(None, 4, 32, 4, 16, 16, None) == moe.MOE_ERR_INVALID_ARG
+    sh = moe.make_shape(64, 32, 4, 2880, 2880)
+    need = moe.moe_workspace_size(sh, moe.WS_LAYER)
+    assert L.moe_layer_forward(16, 16, sh, 16, 16, 16, 16, 16, 16, need - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_layer_forward(16, 16, sh, 16, 16, 16, 16, 16, None, need, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_layer_forward(16, None, sh, 16, 16, 16, 16, 16, 16, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(16, 16, 16, sh, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_permute(16, 16, sh, None, 16, 16, 16, 16, None, 0, None) == moe.MOE_ERR_INVALID_ARG
