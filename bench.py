@@ -45,8 +45,8 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "20b_decode"
 FLUSH_BYTES = 256 << 20
 # kernel launches of one moe_layer_forward call: route, permute (bookkeeping +
-# row gather), expert MLP (gate/up, down), combine
-LAUNCHES_PER_LAYER = 6
+# row gather), expert MLP (tile plan, gate/up GEMM, down GEMM), combine
+LAUNCHES_PER_LAYER = 7
 # dram bytes (read + write) of one moe_expert_mlp call on the default workload,
 # from an ncu capture of the kernels whose source hashes to TRAFFIC_SRC_SHA;
 # reported only while the source is unchanged

@@ -21,7 +21,7 @@ size_t expert_mlp_workspace(const moe_shape& sh);
 moe_status expert_mlp_launch(const uint16_t* x_perm, const int32_t* offsets, const moe_shape& sh,
                              const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
                              const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
-                             cudaStream_t stream);
+                             int32_t* status, cudaStream_t stream);
 moe_status combine_launch(const uint16_t* y_perm, const int32_t* slot_pos, const float* w,
                           const moe_shape& sh, uint16_t* out, cudaStream_t stream);
 
@@ -166,7 +166,7 @@ moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, moe_sh
   moe_status st = check_device();
   if (st != MOE_OK) return st;
   return expert_mlp_launch(x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm, ws,
-                           static_cast<cudaStream_t>(stream));
+                           nullptr, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape shape,
@@ -204,7 +204,7 @@ moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape s
       MOE_OK)
     return st;
   if ((st = expert_mlp_launch(x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm,
-                              at(L.mlp), s)) != MOE_OK)
+                              at(L.mlp), static_cast<int32_t*>(at(L.status)), s)) != MOE_OK)
     return st;
   return combine_launch(y_perm, slot_pos, w, shape, out, s);
 }

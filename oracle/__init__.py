@@ -62,7 +62,8 @@ def _L():
         lib.oracle_combine.argtypes = [vp, vp, vp, i64, i32, i32, vp]
         lib.oracle_layer_forward.argtypes = [vp, vp, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32]
         lib.oracle_layer_forward.restype = i32
-        lib.oracle_layer_tokens.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, vp, i32]
+        lib.oracle_layer_tokens.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, vp,
+                                            vp, i32]
         lib.oracle_layer_tokens.restype = i32
         _lib = lib
     return _lib
@@ -193,8 +194,9 @@ def layer_forward(x, logits, k, wgu_q, wgu_s, wdn_q, wdn_s) -> np.ndarray:
     return out
 
 
-def layer_tokens(x, logits, k, wgu_q, wgu_s, wdn_q, wdn_s, tokens) -> np.ndarray:
-    """Output rows of the selected tokens, computed per token (no permutation)."""
+def layer_tokens(x, logits, k, wgu_q, wgu_s, wdn_q, wdn_s, tokens, want_y: bool = False):
+    """Output rows of the selected tokens, computed per token (no permutation);
+    with want_y also the bf16 expert outputs [len(tokens)][k][D]."""
     xx = _c(x, np.uint16)
     lg = _c(logits, np.float32)
     T, D = xx.shape
@@ -203,11 +205,12 @@ def layer_tokens(x, logits, k, wgu_q, wgu_s, wdn_q, wdn_s, tokens) -> np.ndarray
     tk = _c(np.asarray(tokens), np.int64)
     gq, gs, dq, ds = (_c(a, np.uint8) for a in (wgu_q, wgu_s, wdn_q, wdn_s))
     out = np.empty((tk.size, D), dtype=np.uint16)
+    y = np.empty((tk.size, k, D), dtype=np.uint16) if want_y else None
     rc = _L().oracle_layer_tokens(_p(xx), _p(lg), E, k, D, F, _p(gq), _p(gs), _p(dq), _p(ds),
-                                  _p(tk), tk.size, _p(out), _threads())
+                                  _p(tk), tk.size, _p(out), _p(y) if want_y else None, _threads())
     if rc != 0:
         raise MemoryError("oracle_layer_tokens: allocation failed")
-    return out
+    return (out, y) if want_y else out
 
 
 def quantize_experts(w_bf16: np.ndarray) -> tuple[np.ndarray, np.ndarray]:

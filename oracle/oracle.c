@@ -418,11 +418,12 @@ int oracle_layer_forward(const uint16_t* x, const float* logits, int64_t T, int 
 
 /* the layer for selected tokens only, written per token with no permutation:
  * for token t, route it, run each chosen expert on x[t], mix with the
- * softmax weights.  out_rows[i] is the output row of token tokens[i]. */
+ * softmax weights.  out_rows[i] is the output row of token tokens[i];
+ * y_rows (nullable) receives the bf16 expert outputs [i][j][D]. */
 int oracle_layer_tokens(const uint16_t* x, const float* logits, int E, int k, int D, int F,
                         const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
                         const uint8_t* wdn_s, const int64_t* tokens, int64_t n_tokens,
-                        uint16_t* out_rows, int nthreads) {
+                        uint16_t* out_rows, uint16_t* y_rows, int nthreads) {
   int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n_tokens * k + 1));
   double* w = (double*)malloc(sizeof(double) * (size_t)(n_tokens * k + 1));
   uint16_t* y = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n_tokens * k + 1) * D);
@@ -455,6 +456,8 @@ int oracle_layer_tokens(const uint16_t* x, const float* logits, int E, int k, in
         for (int j = 0; j < k; ++j) acc += w[i * k + j] * oracle_bf16_value(y[(i * k + j) * D + d]);
         out_rows[i * D + d] = oracle_bf16_round(acc);
       }
+    /* optional: the k expert outputs of each token, [n_tokens][k][D] */
+    if (y_rows) memcpy(y_rows, y, sizeof(uint16_t) * (size_t)(n_tokens * k) * D);
     rc = 0;
   }
   free(idx);

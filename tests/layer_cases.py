@@ -37,10 +37,41 @@ def layer_error(got_bits: np.ndarray, ref_bits: np.ndarray) -> tuple[float, floa
     return rel, mx, rms
 
 
-def assert_layer_close(got_bits, ref_bits, what=""):
+def bf16_ulp(bits: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at each element: 2^(exponent - 7) (2^-133 for
+    zero and subnormals)."""
+    e = ((bits.astype(np.int64) >> 7) & 0xFF)
+    return np.ldexp(1.0, (np.maximum(e, 1) - 127 - 7).astype(np.int64))
+
+
+def assert_layer_close(got_bits, ref_bits, what="", y_ulp=None):
+    """Relative Frobenius error <= 5e-3, and per element
+    |got - ref| <= 1e-2 * rms(ref) + ulp(ref) + y_ulp.
+
+    The two ulp terms are the reading of the max-abs bar for a layer whose
+    intermediates and output are bf16: each bf16 rounding point may land on
+    the other neighbour when the library (fp32 accumulation) and the oracle
+    (fp64) see a sum within fp32 error of a rounding boundary.  ulp(ref)
+    covers the final rounding of the output; y_ulp (the largest bf16 ulp of
+    the k expert outputs y_j mixed into the element, whose weights sum to 1)
+    covers a flip of one y_j.  Outputs above ~2.6 rms already have one ulp
+    above 1e-2 * rms, so without these terms the bar would reject any
+    fp32-accumulating implementation.  Differences beyond one ulp of the
+    output must also stay rare (<= 1% of elements)."""
+    got_bits = np.asarray(got_bits, dtype=np.uint16)
+    ref_bits = np.asarray(ref_bits, dtype=np.uint16)
     rel, mx, rms = layer_error(got_bits, ref_bits)
     assert rel <= REL_FRO, f"{what}: relative Frobenius error {rel:.3e} > {REL_FRO}"
-    assert mx <= MAX_ABS_RMS * rms, f"{what}: max abs error {mx:.3e} > {MAX_ABS_RMS} * rms {rms:.3e}"
+    g, r = f64(got_bits), f64(ref_bits)
+    ulp = bf16_ulp(ref_bits)
+    extra = 0.0 if y_ulp is None else np.asarray(y_ulp, dtype=np.float64)
+    excess = np.abs(g - r) - (MAX_ABS_RMS * rms + ulp + extra)
+    worst = int(np.argmax(excess)) if excess.size else 0
+    assert excess.size == 0 or excess.flat[worst] <= 0, (
+        f"{what}: |diff| {abs(g.flat[worst] - r.flat[worst]):.3e} at {worst} exceeds "
+        f"{MAX_ABS_RMS} * rms {rms:.3e} + ulp {ulp.flat[worst]:.3e} (max abs {mx:.3e})")
+    beyond_ulp = float(np.mean(np.abs(g - r) > ulp)) if g.size else 0.0
+    assert beyond_ulp <= 0.01, f"{what}: {beyond_ulp:.2%} of elements differ by more than one ulp"
     return rel, mx, rms
 
 
@@ -103,6 +134,26 @@ def oracle_weights_for(wl: syn.Workload, experts) -> tuple[np.ndarray, ...]:
         q, s = oracle.quantize_experts(syn.w_down(wl, [e]))
         dq[e], ds[e] = q[0], s[0]
     return gq, gs, dq, ds
+
+
+def oracle_layer_with_y(x, lg, k, gq, gs, dq, ds):
+    """The oracle's layer in its step order, returning the output and, per
+    output element, the largest bf16 ulp among the k expert outputs mixed
+    into it."""
+    E = lg.shape[1]
+    idx, w = oracle.route(lg, k)
+    _, offsets, ss, sp = oracle.permute(idx, E)
+    xp = oracle.gather(x, ss, k)
+    _, y = oracle.expert_mlp(xp, offsets, gq, gs, dq, ds, want_h=False)
+    out = oracle.combine(y, sp, w, k)
+    T = x.shape[0]
+    yt = y[sp].reshape(T, k, -1)
+    return out, bf16_ulp(yt).max(axis=1)
+
+
+def oracle_tokens_with_y(x, lg, k, gq, gs, dq, ds, tokens):
+    out, y = oracle.layer_tokens(x, lg, k, gq, gs, dq, ds, tokens, want_y=True)
+    return out, bf16_ulp(y).max(axis=1)
 
 
 def run_layer(L: DeviceLayer) -> torch.Tensor:

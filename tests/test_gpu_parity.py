@@ -12,8 +12,9 @@ import torch
 import mxfp4_quantised_mixture_b200 as moe
 import oracle
 import synthetic as syn
-from layer_cases import (ROUTE_W_ATOL, assert_layer_close, bf16_np, device_layer, layer_error,
-                         oracle_weights_for, run_layer, to_dev_u16)
+from layer_cases import (ROUTE_W_ATOL, assert_layer_close, bf16_np, bf16_ulp, device_layer,
+                         oracle_layer_with_y, oracle_tokens_with_y, oracle_weights_for, run_layer,
+                         to_dev_u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -191,6 +192,7 @@ def test_expert_mlp_and_combine_tiny(dev):
                        L.wgu_s, L.wdn_q, L.wdn_s, h, y, ws)
     torch.cuda.synchronize()
     assert_layer_close(bf16_np(h), oh, "h")
+    # y mixes bf16 h values: a flip of one h moves y by far less than an ulp
     assert_layer_close(bf16_np(y), oy, "y")
     # combine of the oracle's y with fp32 routing weights
     out = torch.empty((wl.T, wl.d_model), dtype=torch.bfloat16, device=dev)
@@ -210,8 +212,8 @@ def test_layer_full_output(dev, name):
     L = device_layer(wl, dev)
     out = bf16_np(run_layer(L))
     gq, gs, dq, ds = oracle_weights_for(wl, range(wl.E))
-    want = oracle.layer_forward(L.host["x"], L.host["logits"], wl.k, gq, gs, dq, ds)
-    assert_layer_close(out, want, name)
+    want, y_ulp = oracle_layer_with_y(L.host["x"], L.host["logits"], wl.k, gq, gs, dq, ds)
+    assert_layer_close(out, want, name, y_ulp)
 
 
 @pytest.mark.parametrize("name", ["20b_prefill", "120b_skewed_prefill"])
@@ -223,8 +225,8 @@ def test_layer_sampled_tokens(dev, name):
     tokens = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 10)]))
     oi, _ = oracle.route(L.host["logits"][tokens], wl.k)
     gq, gs, dq, ds = oracle_weights_for(wl, oi.ravel())
-    want = oracle.layer_tokens(L.host["x"], L.host["logits"], wl.k, gq, gs, dq, ds, tokens)
-    assert_layer_close(out[tokens], want, name)
+    want, y_ulp = oracle_tokens_with_y(L.host["x"], L.host["logits"], wl.k, gq, gs, dq, ds, tokens)
+    assert_layer_close(out[tokens], want, name, y_ulp)
     # properties that hold at any size: finite, and the scale of the output
     o = out.view(np.uint16)
     assert ((o & 0x7F80) != 0x7F80).all()
@@ -237,8 +239,8 @@ def test_layer_odd_shapes(dev, T, D, F, E, k):
     L = device_layer(wl, dev)
     out = bf16_np(run_layer(L))
     gq, gs, dq, ds = oracle_weights_for(wl, range(E))
-    want = oracle.layer_forward(L.host["x"], L.host["logits"], k, gq, gs, dq, ds)
-    assert_layer_close(out, want, f"{T},{D},{F},{E},{k}")
+    want, y_ulp = oracle_layer_with_y(L.host["x"], L.host["logits"], k, gq, gs, dq, ds)
+    assert_layer_close(out, want, f"{T},{D},{F},{E},{k}", y_ulp)
 
 
 def test_layer_all_tokens_on_few_experts(dev):
@@ -251,8 +253,38 @@ def test_layer_all_tokens_on_few_experts(dev):
     L.host["logits"] = lg
     out = bf16_np(run_layer(L))
     gq, gs, dq, ds = oracle_weights_for(wl, range(4))
-    want = oracle.layer_forward(L.host["x"], lg, 4, gq, gs, dq, ds)
-    assert_layer_close(out, want, "hot")
+    want, y_ulp = oracle_layer_with_y(L.host["x"], lg, 4, gq, gs, dq, ds)
+    assert_layer_close(out, want, "hot", y_ulp)
+
+
+@pytest.mark.parametrize("gu_sigma,dn_sigma,x_sigma", [(3e-39, 0.02, 1e36), (0.02, 1e3, 1.0)])
+def test_layer_extreme_scales(dev, gu_sigma, dn_sigma, x_sigma):
+    # scale byte 0 (gate/up weights at the bottom of the bf16 range, decoded
+    # values subnormal) and scale bytes above 128 (large down weights)
+    T, D, F, E, k = 24, 256, 256, 8, 4
+    wl = syn.Workload("scales", T=T, d_model=D, d_ff=F, E=E, k=k, seed=12)
+    x_np = syn.normal_bf16(12, 701, (T, D), sigma=x_sigma)
+    lg_np = syn.logits_custom(12, 702, T, E)
+    gu = syn.normal_bf16(12, 703, (E, 2 * F, D), sigma=gu_sigma)
+    dn = syn.normal_bf16(12, 704, (E, D, F), sigma=dn_sigma)
+    gq, gs, _ = oracle.mxfp4_quantize(gu)
+    dq, ds, _ = oracle.mxfp4_quantize(dn)
+    if gu_sigma < 1e-30:
+        assert (gs == 0).mean() > 0.5
+    else:
+        assert (ds > 128).all()
+    shape = moe.make_shape(T, E, k, D, F)
+    wgu_q = torch.from_numpy(gq).to(dev)
+    wgu_s = torch.from_numpy(gs).to(dev)
+    wdn_q = torch.from_numpy(dq).to(dev)
+    wdn_s = torch.from_numpy(ds).to(dev)
+    out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    ws = moe.alloc_workspace(shape, moe.WS_LAYER, dev)
+    moe.moe_layer_forward(to_dev_u16(x_np, dev), torch.from_numpy(lg_np).to(dev), shape, wgu_q,
+                          wgu_s, wdn_q, wdn_s, out, ws)
+    torch.cuda.synchronize()
+    want, y_ulp = oracle_layer_with_y(x_np, lg_np, k, gq, gs, dq, ds)
+    assert_layer_close(bf16_np(out), want, f"scales {gu_sigma} {dn_sigma}", y_ulp)
 
 
 def test_layer_is_deterministic(dev):
