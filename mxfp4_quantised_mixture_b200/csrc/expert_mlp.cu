@@ -9,22 +9,27 @@
 //
 // One kernel template runs both GEMMs of the MLP.  A CTA owns one tile:
 // 128 weight rows (the MMA's M side) x up to NT routed token rows of one
-// expert (the N side) x the whole reduction axis K.
+// expert (the N side) x the whole reduction axis K, in stages of BK = 64.
 //   * gate/up: the 128 rows are 64 gate rows and the matching 64 up rows,
 //     interleaved in tensor memory (lane 2j = gate j, lane 2j+1 = up j), so
 //     the SwiGLU epilogue pairs neighbouring lanes; output h [S][F] bf16.
 //   * down: 128 rows of the [D][F] matrix; output y_perm [S][D] bf16.
-// Warp roles (64 + 128 * kDecodeGroups threads):
-//   warp 0       TMA producer: packed weight codes (BK/2 bytes per row per
-//                stage), token rows (bf16, 128-byte swizzle) and, once per
-//                tile, the tile's E8M0 scale bytes (bulk copy)
-//   warp 1       tensor-memory owner and MMA issuer: D[128 x NT] (fp32, in
-//                tensor memory) += A[128 x 16] * B[NT x 16]^T per instruction,
-//                A read from tensor memory, B from shared memory
-//   warpgroups   decoders: each thread owns one weight row (its tensor-memory
-//                lane), turns 64 codes per stage into bf16 (exact: the codes
-//                times a power of two) and stores them to an A slot in tensor
-//                memory; after the K loop they run the epilogue.
+// Warp roles (4 + 4 * kDecodeGroups warps):
+//   warp 0       weight producer: the tile's E8M0 scale bytes (one bulk
+//                copy) and per stage the packed codes (TMA, 4 KB) into an
+//                8-deep ring released by the decoders
+//   warp 1       token producer and tensor-memory owner: per stage NT token
+//                rows x 64 bf16 (TMA, 128-byte swizzle) into slot j of a ring
+//                whose slot j pairs with A slot j in tensor memory
+//   warps 2, 3   MMA issuers, taking even and odd stages into two fp32
+//                accumulators in tensor memory (D0, D1); one commit per stage
+//                frees both the token slot and the A slot.  Two issuers keep
+//                the tensor core fed: one thread issues an M=128, N<=64 MMA
+//                only every ~50 cycles and a commit costs a few hundred.
+//   warpgroups   decoders, taking stages round-robin: each thread owns one
+//                weight row (its tensor-memory lane), turns 64 codes per
+//                stage into exact bf16 and writes them to the stage's A slot;
+//                after the K loop they add D0 + D1 and run the epilogue.
 // Decode: code nibble s|m2|m1|m0 is placed as the bf16 bit pattern
 // s<<15 | m2<<8 | m1<<7 | m0<<6, which is the E2M1 value times 2^-126 (code 1
 // lands on the subnormal 2^-127); two byte-table permutes build the high and
@@ -42,22 +47,27 @@
 namespace moe {
 namespace {
 
-constexpr int BK = 64;             // K elements per pipeline stage
-constexpr int BM = 128;            // weight rows per tile (MMA M)
+constexpr int BK = 64;                // K elements per pipeline stage
+constexpr int BM = 128;               // weight rows per tile (MMA M)
 constexpr int W_STAGE = BM * BK / 2;  // packed code bytes per stage
-constexpr int kASlots = 4;         // A stages in tensor memory (32 columns each)
-constexpr int kDecodeGroups = 2;
-constexpr int kThreads = 64 + 128 * kDecodeGroups;
+constexpr int NSW = 8;                // weight ring depth
+constexpr int kDecodeGroups = 3;
+constexpr int kDecWarp0 = 4;
+constexpr int kThreads = 32 * (kDecWarp0 + 4 * kDecodeGroups);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct Tile {
   int e, row0, nrows, pad;
 };
 
-__host__ __device__ constexpr int stages_for(int NT) { return NT <= 64 ? 8 : (NT <= 128 ? 6 : 4); }
-
+// per token-tile width: token/A slots and MMA issuers (tensor memory holds
+// NMMA accumulators of NT columns plus NA A slots of 32 columns)
+__host__ __device__ constexpr int slots_for(int NT) {
+  return NT == 32 ? 6 : (NT == 64 ? 4 : (NT == 128 ? 6 : 4));
+}
+__host__ __device__ constexpr int issuers_for(int NT) { return NT <= 128 ? 2 : 1; }
 __host__ __device__ constexpr int tmem_cols_for(int NT) {
-  return (NT + kASlots * 32) <= 256 ? 256 : 512;
+  return issuers_for(NT) * NT + slots_for(NT) * 32 <= 256 ? 256 : 512;
 }
 
 struct SmemLayout {
@@ -66,12 +76,11 @@ struct SmemLayout {
 
 __host__ __device__ inline SmemLayout smem_layout(int NT, int K) {
   SmemLayout L;
-  const int ns = stages_for(NT);
   L.x_off = 0;
-  L.w_off = L.x_off + ns * NT * 128;
-  L.s_off = L.w_off + ns * W_STAGE;
+  L.w_off = L.x_off + slots_for(NT) * NT * 128;
+  L.s_off = L.w_off + NSW * W_STAGE;
   L.bar_off = L.s_off + ((BM * (K / 32) + 127) / 128) * 128;
-  L.total = L.bar_off + 256;
+  L.total = L.bar_off + 512;
   return L;
 }
 
@@ -132,14 +141,20 @@ __device__ __forceinline__ void abort_cta(volatile int* abort, int32_t* status) 
   record_status(status, MOE_ERR_TIMEOUT);
 }
 
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  const bool r = tc::mbar_wait(bar, parity, abort, kWaitLimitNs);
+  return __all_sync(0xFFFFFFFFu, r);
+}
+
 template <int NT, bool GATE_UP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per SM for narrow tiles
     grouped_mxfp4_gemm(const __grid_constant__ CUtensorMap map_w,
                        const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ scales,
                        const Tile* __restrict__ tiles, const int* __restrict__ n_tiles,
                        int rows_per_expert, int K, int out_ld, uint16_t* __restrict__ out,
                        int32_t* __restrict__ status) {
-  constexpr int NS = stages_for(NT);
+  constexpr int NA = slots_for(NT);
+  constexpr int NMMA = issuers_for(NT);
   constexpr int X_STAGE = NT * 128;
   constexpr int TMEM_COLS = tmem_cols_for(NT);
   constexpr uint32_t IDESC = tc::idesc_bf16_f32(BM, NT);
@@ -153,12 +168,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* wsm = smem + L.w_off;
   uint8_t* ssm = smem + L.s_off;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* full = bars;                 // [NS]  TMA landed (weights + tokens)
-  uint64_t* empty = bars + NS;           // [NS]  stage consumed by decoders and MMA
-  uint64_t* afull = bars + 2 * NS;       // [kASlots] A slot written by decoders
-  uint64_t* aempty = afull + kASlots;    // [kASlots] A slot read by the MMA
-  uint64_t* sbar = aempty + kASlots;     // scales landed
-  uint64_t* dfull = sbar + 1;            // accumulator complete
+  uint64_t* wfull = bars;              // [NSW] weight codes landed
+  uint64_t* wempty = wfull + NSW;      // [NSW] weight codes read by the decoders
+  uint64_t* xfull = wempty + NSW;      // [NA]  token rows landed
+  uint64_t* afull = xfull + NA;        // [NA]  A slot written by the decoders
+  uint64_t* consumed = afull + NA;     // [NA]  MMA done with token slot + A slot
+  uint64_t* sbar = consumed + NA;      // scales landed
+  uint64_t* dfull = sbar + 1;          // accumulators complete (one commit per issuer)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(dfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -169,16 +185,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kscale = K / 32;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 4 + 1);
+    for (int s = 0; s < NSW; ++s) {
+      tc::mbar_init(&wfull[s], 1);
+      tc::mbar_init(&wempty[s], 4);
     }
-    for (int j = 0; j < kASlots; ++j) {
+    for (int j = 0; j < NA; ++j) {
+      tc::mbar_init(&xfull[j], 1);
       tc::mbar_init(&afull[j], 4);
-      tc::mbar_init(&aempty[j], 1);
+      tc::mbar_init(&consumed[j], 1);
     }
     tc::mbar_init(sbar, 1);
-    tc::mbar_init(dfull, 1);
+    tc::mbar_init(dfull, NMMA);
     *abort_flag = 0;
     tc::fence_mbar_init();
     tc::tma_prefetch_desc(&map_w);
@@ -192,78 +209,99 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_d = tmem;       // accumulator: columns [0, NT)
-  const uint32_t tmem_a = tmem + NT;  // A slots: columns [NT, NT + 32 * kASlots)
+  const uint32_t tmem_a = tmem + NMMA * NT;  // A slots follow the accumulators
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // -------------------------------------------------- weight producer
     if (lane == 0) {
       const int r0 = GATE_UP ? mt * 64 : mt * BM;
       const int64_t srow = static_cast<int64_t>(tile.e) * rows_per_expert;
-      uint32_t sbytes;
       if (GATE_UP) {
         const uint32_t half = 64u * kscale;
-        sbytes = 2 * half;
-        tc::mbar_arrive_expect_tx(sbar, sbytes);
+        tc::mbar_arrive_expect_tx(sbar, 2 * half);
         const int F = rows_per_expert / 2;
         tc::bulk_load(ssm, scales + (srow + r0) * kscale, half, sbar);
         tc::bulk_load(ssm + half, scales + (srow + F + r0) * kscale, half, sbar);
       } else {
-        const int nrows = min(BM, rows_per_expert - r0);
-        sbytes = static_cast<uint32_t>(nrows) * kscale;
-        tc::mbar_arrive_expect_tx(sbar, sbytes);
-        tc::bulk_load(ssm, scales + (srow + r0) * kscale, sbytes, sbar);
+        const uint32_t bytes = static_cast<uint32_t>(min(BM, rows_per_expert - r0)) * kscale;
+        tc::mbar_arrive_expect_tx(sbar, bytes);
+        tc::bulk_load(ssm, scales + (srow + r0) * kscale, bytes, sbar);
       }
       int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % NS, n = kb / NS;
-        if (n > 0 && !tc::mbar_wait(&empty[s], (n - 1) & 1, abort_flag, kWaitLimitNs)) {
+        const int s = kb % NSW, n = kb / NSW;
+        if (n > 0 && !tc::mbar_wait(&wempty[s], (n - 1) & 1, abort_flag, kWaitLimitNs)) {
           abort_cta(abort_flag, status);
           break;
         }
-        tc::mbar_arrive_expect_tx(&full[s], W_STAGE + X_STAGE);
+        tc::mbar_arrive_expect_tx(&wfull[s], W_STAGE);
         uint8_t* wdst = wsm + s * W_STAGE;
         if (GATE_UP) {
           const int F = rows_per_expert / 2;
-          tc::tma_load_3d(wdst, &map_w, &full[s], kb * (BK / 2), r0, tile.e);
-          tc::tma_load_3d(wdst + W_STAGE / 2, &map_w, &full[s], kb * (BK / 2), F + r0, tile.e);
+          tc::tma_load_3d(wdst, &map_w, &wfull[s], kb * (BK / 2), r0, tile.e);
+          tc::tma_load_3d(wdst + W_STAGE / 2, &map_w, &wfull[s], kb * (BK / 2), F + r0, tile.e);
         } else {
-          tc::tma_load_3d(wdst, &map_w, &full[s], kb * (BK / 2), r0, tile.e);
+          tc::tma_load_3d(wdst, &map_w, &wfull[s], kb * (BK / 2), r0, tile.e);
         }
-        tc::tma_load_2d(xs + s * X_STAGE, &map_x, &full[s], kb * BK, tile.row0);
         ++issued;
       }
       // drain: every copy this thread issued has landed before the CTA exits
-      for (int kb = max(0, issued - NS); kb < issued; ++kb)
-        tc::mbar_wait(&full[kb % NS], (kb / NS) & 1, abort_flag, kWaitLimitNs / 8);
+      for (int kb = max(0, issued - NSW); kb < issued; ++kb)
+        tc::mbar_wait(&wfull[kb % NSW], (kb / NSW) & 1, abort_flag, kWaitLimitNs / 8);
       tc::mbar_wait(sbar, 0, abort_flag, kWaitLimitNs / 8);
     }
   } else if (warp == 1) {
-    // --------------------------------------------------------------- MMA
+    // --------------------------------------------------- token producer
     if (lane == 0) {
+      int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % NS, j = kb % kASlots;
-        if (!tc::mbar_wait(&full[s], (kb / NS) & 1, abort_flag, kWaitLimitNs) ||
-            !tc::mbar_wait(&afull[j], (kb / kASlots) & 1, abort_flag, kWaitLimitNs)) {
+        const int j = kb % NA, n = kb / NA;
+        if (n > 0 && !tc::mbar_wait(&consumed[j], (n - 1) & 1, abort_flag, kWaitLimitNs)) {
+          abort_cta(abort_flag, status);
+          break;
+        }
+        tc::mbar_arrive_expect_tx(&xfull[j], X_STAGE);
+        tc::tma_load_2d(xs + j * X_STAGE, &map_x, &xfull[j], kb * BK, tile.row0);
+        ++issued;
+      }
+      for (int kb = max(0, issued - NA); kb < issued; ++kb)
+        tc::mbar_wait(&xfull[kb % NA], (kb / NA) & 1, abort_flag, kWaitLimitNs / 8);
+    }
+  } else if (warp < kDecWarp0) {
+    // ---------------------------------------------------------- MMA issuers
+    const int mi = warp - 2;  // this issuer's stages: kb = mi, mi + NMMA, ...
+    if (lane == 0 && mi < NMMA) {
+      const uint32_t tmem_d = tmem + mi * NT;
+      int done = 0;
+      for (int kb = mi; kb < KB; kb += NMMA) {
+        const int j = kb % NA;
+        const uint32_t par = (kb / NA) & 1;
+        if (!tc::mbar_wait(&xfull[j], par, abort_flag, kWaitLimitNs) ||
+            !tc::mbar_wait(&afull[j], par, abort_flag, kWaitLimitNs)) {
           abort_cta(abort_flag, status);
           break;
         }
         tc::tc_fence_after();
-        const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(xs + s * X_STAGE));
+        const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(xs + j * X_STAGE));
 #pragma unroll
         for (int i = 0; i < BK / 16; ++i)
           tc::mma_bf16_ts(tmem_d, tmem_a + j * 32 + i * 8, bdesc + static_cast<uint64_t>(i * 2),
-                          IDESC, (kb | i) != 0);
-        tc::mma_commit(&aempty[j]);
-        tc::mma_commit(&empty[s]);
+                          IDESC, (done | i) != 0);
+        tc::mma_commit(&consumed[j]);
+        ++done;
       }
-      tc::mma_commit(dfull);  // also on abort: completes once issued MMAs finish
+      // completes once every MMA this thread issued has finished (also on
+      // abort); an issuer with no stage (K = 64) only arrives
+      if (done > 0)
+        tc::mma_commit(dfull);
+      else
+        tc::mbar_arrive(dfull);
     }
   } else {
     // ----------------------------------------------------------- decoders
-    const int g = (warp - 2) >> 2;  // decode group
-    const int q = warp & 3;         // tensor-memory lane quarter of this warp
-    const int m = q * 32 + lane;    // tensor-memory lane = weight row in tile
+    const int g = (warp - kDecWarp0) >> 2;  // decode group
+    const int q = warp & 3;                 // tensor-memory lane quarter of this warp
+    const int m = q * 32 + lane;            // tensor-memory lane = weight row in tile
     int wrow, srow_s, rot;
     if (GATE_UP) {
       wrow = (m & 1) * (W_STAGE / 2) + (m >> 1) * (BK / 2);
@@ -275,15 +313,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       rot = (m >> 2) & 1;
     }
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    bool ok = tc::mbar_wait(sbar, 0, abort_flag, kWaitLimitNs);
+    bool ok = warp_wait(sbar, 0, abort_flag);
     if (!ok) abort_cta(abort_flag, status);
     // rows past the end of the expert's matrix (last down tile) read no scales
     const bool row_live = GATE_UP || (mt * BM + m < rows_per_expert);
     const uint8_t* my_scales = ssm + srow_s * kscale;
     for (int kb = g; ok && kb < KB; kb += kDecodeGroups) {
-      const int s = kb % NS, j = kb % kASlots;
-      if (!tc::mbar_wait(&full[s], (kb / NS) & 1, abort_flag, kWaitLimitNs)) {
+      const int s = kb % NSW, j = kb % NA;
+      if (!warp_wait(&wfull[s], (kb / NSW) & 1, abort_flag)) {
         abort_cta(abort_flag, status);
+        ok = false;
         break;
       }
       const uint8_t* src = wsm + s * W_STAGE + wrow;
@@ -299,32 +338,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         s1 = my_scales[2 * kb + 1];
       }
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty[s]);
-      const int use = kb / kASlots;
-      if (use > 0 && !tc::mbar_wait(&aempty[j], (use - 1) & 1, abort_flag, kWaitLimitNs)) {
+      if (lane == 0) tc::mbar_arrive(&wempty[s]);
+      uint32_t o0[16], o1[16];
+      decode32(p0, s0, o0);
+      decode32(p1, s1, o1);
+      const int use = kb / NA;
+      if (use > 0 && !warp_wait(&consumed[j], (use - 1) & 1, abort_flag)) {
         abort_cta(abort_flag, status);
+        ok = false;
         break;
       }
       tc::tc_fence_after();
-      uint32_t o[16];
-      decode32(p0, s0, o);
-      tc::tmem_st16(tmem_a + lane_base + j * 32, o);
-      decode32(p1, s1, o);
-      tc::tmem_st16(tmem_a + lane_base + j * 32 + 16, o);
+      tc::tmem_st16(tmem_a + lane_base + j * 32, o0);
+      tc::tmem_st16(tmem_a + lane_base + j * 32 + 16, o1);
       tc::tmem_st_wait();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&afull[j]);
     }
     // ---------------------------------------------------------- epilogue
-    ok = ok && !*abort_flag && tc::mbar_wait(dfull, 0, abort_flag, kWaitLimitNs);
+    ok = ok && warp_wait(dfull, 0, abort_flag) && *abort_flag == 0;
+    const int used = KB < NMMA ? KB : NMMA;  // accumulators that hold a partial sum
     if (ok) {
       tc::tc_fence_after();
-      uint8_t* stg = xs;  // every stage has been consumed: reuse as staging
+      uint8_t* stg = xs;  // every token slot has been consumed: reuse as staging
       for (int c = g * 16; c < NT; c += 16 * kDecodeGroups) {
+        float v[16];
         uint32_t r[16];
-        tc::tmem_ld16(tmem_d + lane_base + c, r);
+        tc::tmem_ld16(tmem + lane_base + c, r);
         tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+        if (used > 1) {
+          tc::tmem_ld16(tmem + NT + lane_base + c, r);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += __uint_as_float(r[i]);  // D0 + D1, fixed order
+        }
         if (GATE_UP) {
           // even lane: gate row f, odd lane: up row f (f = m >> 1); the even
           // lane finishes tokens c..c+7, the odd lane tokens c+8..c+15
@@ -332,12 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint16_t hv[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float mine_lo = __uint_as_float(r[i]);
-            const float mine_hi = __uint_as_float(r[8 + i]);
-            const float send = up ? mine_lo : mine_hi;
+            const float send = up ? v[i] : v[8 + i];
             const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-            const float gv = up ? recv : mine_lo;
-            const float uv = up ? mine_hi : recv;
+            const float gv = up ? recv : v[i];
+            const float uv = up ? v[8 + i] : recv;
             const float silu = gv / (1.0f + expf(-gv));
             hv[i] = f32_to_bf16_rne(silu * uv);
           }
@@ -349,15 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           uint16_t* st16 = reinterpret_cast<uint16_t*>(stg);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            st16[(c + i) * BM + m] = f32_to_bf16_rne(__uint_as_float(r[i]));
+          for (int i = 0; i < 16; ++i) st16[(c + i) * BM + m] = f32_to_bf16_rne(v[i]);
         }
       }
     }
     // all decoder warps meet before the coalesced stores
     asm volatile("bar.sync 1, %0;" ::"r"(128 * kDecodeGroups));
     if (ok && !*abort_flag) {
-      const int tid = threadIdx.x - 64;
+      const int tid = threadIdx.x - kDecWarp0 * 32;
       const int nthr = 128 * kDecodeGroups;
       if (GATE_UP) {
         // h rows: 64 features (128 bytes = 8 x 16 B) per token
@@ -480,6 +527,9 @@ int choose_nt(const moe_shape& sh) {
   const int64_t want = 2 * ((S + sh.E - 1) / sh.E);
   int nt = 32;
   while (nt < want && nt < 256) nt *= 2;
+  // the tile must fit shared memory together with the scale bytes of K
+  const int K = sh.d_model > sh.d_ff ? sh.d_model : sh.d_ff;
+  while (nt > 32 && smem_layout(nt, K).total + 1024 > 227 * 1024) nt /= 2;
   return nt;
 }
 
@@ -488,6 +538,7 @@ moe_status launch_gemm(const CUtensorMap& mw, const CUtensorMap& mx, const uint8
                        const Tile* tiles, const int* n_tiles, int grid_x, int grid_y, int R, int K,
                        int out_ld, uint16_t* out, int32_t* status, cudaStream_t stream) {
   const int smem = smem_layout(NT, K).total + 1024;
+  if (smem > 227 * 1024) return MOE_ERR_SHAPE;
   auto kern = grouped_mxfp4_gemm<NT, GATE_UP>;
   static bool attr_done = false;
   static int attr_smem = 0;
