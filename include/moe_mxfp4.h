@@ -207,6 +207,35 @@ MOE_API moe_status moe_layer_forward(const uint16_t* x, const float* logits,
                              const uint8_t* wdn_s, uint16_t* out, void* ws,
                              size_t ws_bytes, moe_stream stream);
 
+/* moe_layer_forward_static -- moe_layer_forward without a caller-supplied
+ * workspace.  The pages have no counterpart: this entry exists for callers
+ * that cannot allocate device memory themselves -- code embedded in a host
+ * application or framework that owns every device allocation and hands out
+ * no allocator, plug-ins that may only use buffers they are given, or paths
+ * where a cudaMalloc (which may synchronise the device) is not acceptable.
+ * It allocates nothing and calls no allocating routine: the intermediates
+ * live in a device array of MOE_STATIC_SCRATCH_BYTES (16 MiB) inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress, with the device current); make that first call
+ * before any stream capture.
+ *   Arguments, layouts and errors are those of moe_layer_forward, minus the
+ *   workspace.  A shape with moe_workspace_size(shape, 2) above
+ *   MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_WORKSPACE before
+ *   anything runs (at d_model = d_ff = 2880 and k = 4 that allows T <= 240).
+ *   Every call uses the same array, and the array keeps the previous call's
+ *   contents: each call clears the part that must start at zero (the device
+ *   status word) and overwrites the rest before reading it.  Calls that can
+ *   overlap on the GPU (other streams, other threads) race on the array and
+ *   must be serialised by the caller; the device status word is not
+ *   readable through this entry (use moe_layer_forward when it must be).  */
+#define MOE_STATIC_SCRATCH_BYTES (16u << 20)
+MOE_API moe_status moe_layer_forward_static(const uint16_t* x, const float* logits,
+                                            moe_shape shape, const uint8_t* wgu_q,
+                                            const uint8_t* wgu_s, const uint8_t* wdn_q,
+                                            const uint8_t* wdn_s, uint16_t* out,
+                                            moe_stream stream);
+
 /* moe_workspace_size -- bytes of device workspace a call needs.
  * which: 0 = moe_permute, 1 = moe_expert_mlp, 2 = moe_layer_forward.
  * Returns 0 for an unsupported shape or an unknown `which`.  Host only.  */

@@ -61,6 +61,8 @@ def _load() -> ctypes.CDLL:
     lib.moe_combine.restype = st
     lib.moe_layer_forward.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_layer_forward.restype = st
+    lib.moe_layer_forward_static.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp]
+    lib.moe_layer_forward_static.restype = st
     lib.moe_workspace_size.argtypes = [moe_shape, ctypes.c_int]
     lib.moe_workspace_size.restype = sz
     lib.moe_status_string.argtypes = [st]
@@ -149,6 +151,18 @@ def moe_layer_forward(x, logits, shape: moe_shape, wgu_q, wgu_s, wdn_q, wdn_s, o
                                                       _p(ws), _nbytes(ws), _s(stream)))
 
 
+STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def moe_layer_forward_static(x, logits, shape: moe_shape, wgu_q, wgu_s, wdn_q, wdn_s, out,
+                             stream=None) -> None:
+    """moe_layer_forward with the intermediates in the library's own 16 MiB
+    device array (for callers that cannot allocate); see the C header."""
+    _check("moe_layer_forward_static",
+           lib.moe_layer_forward_static(_p(x), _p(logits), shape, _p(wgu_q), _p(wgu_s), _p(wdn_q),
+                                        _p(wdn_s), _p(out), _s(stream)))
+
+
 def alloc_workspace(shape: moe_shape, which: int, device="cuda"):
     """A device byte tensor of moe_workspace_size(shape, which) bytes (at least 256)."""
     import torch
@@ -158,5 +172,6 @@ def alloc_workspace(shape: moe_shape, which: int, device="cuda"):
 
 
 __all__ = ["moe_shape", "make_shape", "MoeError", "mxfp4_quantize", "moe_route", "moe_permute",
-           "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_workspace_size",
+           "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_layer_forward_static",
+           "moe_workspace_size",
            "moe_status_string", "alloc_workspace", "lib", "LIB_PATH"]
