@@ -49,8 +49,8 @@ LAUNCHES_PER_LAYER = 7
 # dram bytes (read + write) of one moe_expert_mlp call on the default workload,
 # from an ncu capture of the kernels whose source hashes to TRAFFIC_SRC_SHA;
 # reported only while the source is unchanged
-TRAFFIC_BYTES = None
-TRAFFIC_SRC_SHA = None
+TRAFFIC_BYTES = 438428672  # gate/up 283.63 + 7.64 MB, down 142.56 + 4.60 MB (read + write)
+TRAFFIC_SRC_SHA = "ba748cdc430adb23"
 
 
 def parse():
@@ -228,6 +228,28 @@ def config_dict(wl):
             "parallelism": "replica per GPU"}
 
 
+# ---------------------------------------------------------- rank helpers
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of `value` over all ranks of the default process group (the value
+    itself when there is none)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job tokens/s: every rank ran `steps` steps of its own batch; the
+    job took as long as the slowest rank."""
+    return world * tokens_per_rank * steps / (max_total_ms / 1e3)
+
+
 # -------------------------------------------------------------------- ours
 
 
@@ -313,13 +335,9 @@ def run_ours(args):
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1e3)
+    value = job_throughput(world, T, args.steps, total_ms)
 
     # ---- roofline of the grouped expert MLP: the same step through the
     #      individual calls, with events around moe_expert_mlp
@@ -372,11 +390,7 @@ def run_ours(args):
         out_host.copy_(out, non_blocking=True)
         e_ends[i].record(stream)
         e_ends[i].synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps, dev)
     e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": x_host.numel() * 2 + lg_host.numel() * 4,
            "d2h_bytes_per_step": out_host.numel() * 2}
