@@ -43,14 +43,15 @@ METRIC = "MoE-layer tokens/s on 1 B200; % of roofline (HBM GB/s decode, TC TFLOP
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "20b_decode"
 FLUSH_BYTES = 256 << 20
-# kernel launches of one moe_layer_forward call: route, permute (bookkeeping +
-# row gather), expert MLP (tile plan, gate/up GEMM, down GEMM), combine
-LAUNCHES_PER_LAYER = 7
+# kernel launches of one moe_layer_forward call on the default (decode)
+# workload: route, permute (bookkeeping + row gather), expert MLP (tile plan,
+# activation split, gate/up GEMM, intermediate split, down GEMM), combine
+LAUNCHES_PER_LAYER = 9
 # dram bytes (read + write) of one moe_expert_mlp call on the default workload,
 # from an ncu capture of the kernels whose source hashes to TRAFFIC_SRC_SHA;
 # reported only while the source is unchanged
-TRAFFIC_BYTES = 438428672  # gate/up 283.63 + 7.64 MB, down 142.56 + 4.60 MB (read + write)
-TRAFFIC_SRC_SHA = "ba748cdc430adb23"
+TRAFFIC_BYTES = None
+TRAFFIC_SRC_SHA = None
 
 
 def parse():

@@ -55,7 +55,9 @@
  *     (`d_status`, or the first 4 bytes of the workspace); the caller reads
  *     it after synchronising.  Kernels never trap or assert.
  *   - Calls on different streams with different workspaces are independent.
- *   - Every device pointer must be 16-byte aligned.
+ *   - Every device pointer must be 16-byte aligned; the packed weight code
+ *     arrays (wgu_q, wdn_q) 32-byte aligned (the tensor-memory copy engine
+ *     reads them in the one-byte-per-code layout the tensor core takes).
  */
 #ifndef MOE_MXFP4_H
 #define MOE_MXFP4_H
@@ -80,7 +82,7 @@ typedef enum {
 
 /* Shape of one MoE layer call.
  * Supported: 1 <= T <= 1<<20, 1 <= E <= 256, 1 <= k <= min(E, 8),
- * D and F multiples of 64 in [64, 16384], T*k < 2^31.                    */
+ * D and F multiples of 64 in [128, 16384], T*k < 2^31.                   */
 typedef struct {
   int32_t T;
   int32_t E;
@@ -169,7 +171,8 @@ MOE_API moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x,
  *   y_perm[r] = bf16_rne(h[r] . Wd_e^T)
  *   x_perm  in   [S][D] bf16
  *   offsets in   [E+1] as produced by moe_permute
- *   wgu_q/s in   MXFP4 [E][2F][D]; wdn_q/s in MXFP4 [E][D][F]
+ *   wgu_q/s in   MXFP4 [E][2F][D]; wdn_q/s in MXFP4 [E][D][F]; the code
+ *                arrays wgu_q and wdn_q 32-byte aligned
  *   h       out  [S][F] bf16 (caller-owned intermediate)
  *   y_perm  out  [S][D] bf16
  *   ws      in   device workspace of moe_workspace_size(shape, 1) bytes
@@ -222,7 +225,8 @@ MOE_API moe_status moe_layer_forward(const uint16_t* x, const float* logits,
  *   Arguments, layouts and errors are those of moe_layer_forward, minus the
  *   workspace.  A shape with moe_workspace_size(shape, 2) above
  *   MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_WORKSPACE before
- *   anything runs (at d_model = d_ff = 2880 and k = 4 that allows T <= 240).
+ *   anything runs (at d_model = d_ff = 2880, E = 32 and k = 4 that allows
+ *   T <= 113).
  *   Every call uses the same array, and the array keeps the previous call's
  *   contents: each call clears the part that must start at zero (the device
  *   status word) and overwrites the rest before reading it.  Calls that can

@@ -104,8 +104,8 @@ bool shape_ok(const moe_shape& s) {
   if (s.T < 0 || s.T > (1 << 20)) return false;
   if (s.E < 1 || s.E > 256) return false;
   if (s.k < 1 || s.k > 8 || s.k > s.E) return false;
-  if (s.d_model < 64 || s.d_model > 16384 || (s.d_model % 64) != 0) return false;
-  if (s.d_ff < 64 || s.d_ff > 16384 || (s.d_ff % 64) != 0) return false;
+  if (s.d_model < 128 || s.d_model > 16384 || (s.d_model % 64) != 0) return false;
+  if (s.d_ff < 128 || s.d_ff > 16384 || (s.d_ff % 64) != 0) return false;
   if (static_cast<int64_t>(s.T) * s.k >= (int64_t(1) << 31)) return false;
   return true;
 }
@@ -161,6 +161,7 @@ moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, moe_sh
   const void* ptrs[] = {x_perm, offsets, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (!aligned32(wgu_q) || !aligned32(wdn_q)) return MOE_ERR_INVALID_ARG;
   const size_t need = expert_mlp_workspace(shape);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return MOE_ERR_WORKSPACE;
   moe_status st = check_device();
@@ -179,6 +180,7 @@ moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape s
   const void* ptrs[] = {x, logits, wgu_q, wgu_s, wdn_q, wdn_s, out};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (!aligned32(wgu_q) || !aligned32(wdn_q)) return MOE_ERR_INVALID_ARG;
   const LayerWs L = layer_ws(shape);
   if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   moe_status st = check_device();

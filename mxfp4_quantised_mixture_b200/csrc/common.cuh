@@ -34,6 +34,7 @@ __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
 // ------------------------------------------------------------ host helpers
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

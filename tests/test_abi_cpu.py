@@ -68,6 +68,8 @@ def test_workspace_size_is_host_only_and_monotone():
     (64, 4, 5, 2880, 2880),      # k > E
     (64, 32, 4, 2880, 2890),     # F not a multiple of 64
     (64, 32, 4, 32, 2880),       # D too small
+    (64, 32, 4, 64, 2880),       # D below the 128-code weight window
+    (64, 32, 4, 2880, 64),       # F below the 128-code weight window
     (-1, 32, 4, 2880, 2880),     # T < 0
 ])
 def test_bad_shapes_rejected_before_the_device(shape):
@@ -88,8 +90,15 @@ def test_bad_arguments_rejected_before_the_device():
     assert L.moe_route(None, 4, 32, 4, 16, 16, None) == moe.MOE_ERR_INVALID_ARG
     sh = moe.make_shape(64, 32, 4, 2880, 2880)
     need = moe.moe_workspace_size(sh, moe.WS_LAYER)
-    assert L.moe_layer_forward(16, 16, sh, 16, 16, 16, 16, 16, 16, need - 1, None) == moe.MOE_ERR_WORKSPACE
-    assert L.moe_layer_forward(16, 16, sh, 16, 16, 16, 16, 16, None, need, None) == moe.MOE_ERR_WORKSPACE
-    assert L.moe_layer_forward(16, None, sh, 16, 16, 16, 16, 16, 16, need, None) == moe.MOE_ERR_INVALID_ARG
+    # weight code arrays at 32-byte addresses, everything else at 16
+    assert L.moe_layer_forward(16, 16, sh, 32, 16, 32, 16, 16, 16, need - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_layer_forward(16, 16, sh, 32, 16, 32, 16, 16, None, need, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_layer_forward(16, None, sh, 32, 16, 32, 16, 16, 16, need, None) == moe.MOE_ERR_INVALID_ARG
+    # a code array only 16-byte aligned is refused
+    assert L.moe_layer_forward(16, 16, sh, 48, 16, 32, 16, 16, 16, need, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_forward(16, 16, sh, 32, 16, 48, 16, 16, 16, need, None) == moe.MOE_ERR_INVALID_ARG
+    mlp = moe.moe_workspace_size(sh, moe.WS_EXPERT_MLP)
+    assert L.moe_expert_mlp(16, 16, sh, 48, 16, 32, 16, 16, 16, 16, mlp, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_mlp(16, 16, sh, 32, 16, 32, 16, 16, 16, 16, mlp - 1, None) == moe.MOE_ERR_WORKSPACE
     assert L.moe_combine(16, 16, 16, sh, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_permute(16, 16, sh, None, 16, 16, 16, 16, None, 0, None) == moe.MOE_ERR_INVALID_ARG

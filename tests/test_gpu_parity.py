@@ -124,7 +124,7 @@ def test_route_odd_shapes_and_ties(dev, T, E, k):
 def _gpu_permute(idx_np, x_np, E, D, dev):
     T, k = idx_np.shape
     S = T * k
-    sh = moe.make_shape(T, E, k, D, 64)
+    sh = moe.make_shape(T, E, k, D, 128)
     idx = torch.from_numpy(idx_np).to(dev)
     x = to_dev_u16(x_np, dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
@@ -232,7 +232,7 @@ def test_layer_sampled_tokens(dev, name):
     assert ((o & 0x7F80) != 0x7F80).all()
 
 
-@pytest.mark.parametrize("T,D,F,E,k", [(1, 64, 64, 4, 4), (3, 192, 320, 8, 2), (33, 256, 128, 16, 4),
+@pytest.mark.parametrize("T,D,F,E,k", [(1, 128, 128, 4, 4), (3, 192, 320, 8, 2), (33, 256, 128, 16, 4),
                                         (70, 128, 256, 64, 8), (17, 2880, 2880, 4, 1)])
 def test_layer_odd_shapes(dev, T, D, F, E, k):
     wl = syn.Workload("odd", T=T, d_model=D, d_ff=F, E=E, k=k, seed=3)
