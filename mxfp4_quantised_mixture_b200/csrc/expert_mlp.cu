@@ -68,7 +68,8 @@
 namespace moe {
 namespace {
 
-constexpr int BKS = 128;            // K elements per stage
+constexpr int BKS = 128;            // K elements per window (one 128-byte swizzle row of codes)
+constexpr int WPS = 2;              // windows per pipeline stage
 constexpr int BN = 128;             // weight rows per work item (MMA N)
 constexpr int MM = 128;             // MMA M: token piece rows
 constexpr int W_SMEM = BN * BKS;    // one byte per code in shared memory
@@ -76,7 +77,7 @@ constexpr int W_TX = BN * BKS / 2;  // bytes the stage's weight copy reads
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (6 + kEpiWarps);
 constexpr int kMaxStages = 12;      // copy ring depth limit (stage slot s also owns scale slot s)
-constexpr int kSlotCols = 8;        // per stage: 4 token-scale + 4 weight-scale columns
+constexpr int kSlotCols = 8 * WPS;  // per stage and window: 4 token-scale + 4 weight-scale columns
 constexpr int kTmemCols = 512;      // two accumulators of BN columns, then the scale slots
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -93,9 +94,9 @@ struct SmemLayout {
 
 __host__ __device__ inline SmemLayout smem_layout(int NT, int NS, int NB, int K) {
   SmemLayout L;
-  L.x_off = 0;  // token ring first: a stage's 128-row MMA view runs on into the weight ring
-  L.w_off = NS * 2 * NT * BKS;
-  L.a_off = L.w_off + NS * W_SMEM;
+  L.x_off = 0;  // token ring first: a window's 128-row MMA view runs on into the weight ring
+  L.w_off = NS * WPS * 2 * NT * BKS;
+  L.a_off = L.w_off + NS * WPS * W_SMEM;
   L.wsc_bytes = ((BN * (K / 32)) + 127) / 128 * 128;
   L.aux_bytes = L.wsc_bytes + ((K + BKS - 1) / BKS) * 2 * NT * 4;
   L.bar_off = L.a_off + NB * L.aux_bytes;
@@ -178,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nstg = (K + BKS - 1) / BKS;
+  const int nwin = (K + BKS - 1) / BKS;    // 128-K windows
+  const int nstg = (nwin + WPS - 1) / WPS;  // pipeline stages of WPS windows
   const int kscale = K / 32;
 
   if (threadIdx.x == 0) {
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (use > 0 && !wait1(&sfree[b], (use - 1) & 1, abort_flag, status)) break;
         const int64_t erow = static_cast<int64_t>(tile.e) * rows_per_expert;
         uint8_t* sdst = aux + b * L.aux_bytes;
-        const uint32_t wbytes = static_cast<uint32_t>(nstg) * XR * 4;
+        const uint32_t wbytes = static_cast<uint32_t>(nwin) * XR * 4;
         if (GATE_UP) {
           const int f0 = mt * (BN / 2);
           const uint32_t bytes = static_cast<uint32_t>(min(BN / 2, F - f0)) * kscale;
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mbar_arrive_expect_tx(&sbar[b], bytes + wbytes);
           tc::bulk_load(sdst, scales + (erow + d0) * kscale, bytes, &sbar[b]);
         }
-        tc::bulk_load(sdst + L.wsc_bytes, sfx_words + static_cast<int64_t>(t) * nstg * XR, wbytes,
+        tc::bulk_load(sdst + L.wsc_bytes, sfx_words + static_cast<int64_t>(t) * nwin * XR, wbytes,
                       &sbar[b]);
         const int wrow = GATE_UP ? mt * (BN / 2) : mt * BN;
         for (int st = 0; st < nstg; ++st, ++g) {
@@ -248,21 +250,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const int k0 = stage_k0(st, K);
-          tc::mbar_arrive_expect_tx(&full[s_slot], W_TX + X_BYTES);
-          uint8_t* wdst = wsm + s_slot * W_SMEM;
-          if (k0 == st * BKS) {
-            if (GATE_UP)
-              tc::tma_load_5d(wdst, &map_w, &full[s_slot], 0, st, 0, wrow, tile.e);
-            else
-              tc::tma_load_4d(wdst, &map_w, &full[s_slot], 0, st, wrow, tile.e);
-          } else {
-            if (GATE_UP)
-              tc::tma_load_4d(wdst, &map_w_tail, &full[s_slot], 0, 0, wrow, tile.e);
-            else
-              tc::tma_load_3d(wdst, &map_w_tail, &full[s_slot], 0, wrow, tile.e);
+          const int w0 = st * WPS;
+          const int nv = min(WPS, nwin - w0);
+          tc::mbar_arrive_expect_tx(&full[s_slot], nv * (W_TX + X_BYTES));
+          for (int v = 0; v < nv; ++v) {
+            const int w = w0 + v;
+            const int k0 = stage_k0(w, K);
+            uint8_t* wdst = wsm + (s_slot * WPS + v) * W_SMEM;
+            if (k0 == w * BKS) {
+              if (GATE_UP)
+                tc::tma_load_5d(wdst, &map_w, &full[s_slot], 0, w, 0, wrow, tile.e);
+              else
+                tc::tma_load_4d(wdst, &map_w, &full[s_slot], 0, w, wrow, tile.e);
+            } else {
+              if (GATE_UP)
+                tc::tma_load_4d(wdst, &map_w_tail, &full[s_slot], 0, 0, wrow, tile.e);
+              else
+                tc::tma_load_3d(wdst, &map_w_tail, &full[s_slot], 0, wrow, tile.e);
+            }
+            tc::tma_load_2d(xs + (s_slot * WPS + v) * X_BYTES, &map_x, &full[s_slot], k0, t * XR);
           }
-          tc::tma_load_2d(xs + s_slot * X_BYTES, &map_x, &full[s_slot], k0, t * XR);
           if (++s_slot == NS) {
             s_slot = 0;
             s_phase ^= 1u;
@@ -287,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true, any = false;
       const uint64_t xdesc0 = tc::smem_desc_sw128(tc::smem_u32(xs));
       const uint64_t wdesc0 = tc::smem_desc_sw128(tc::smem_u32(wsm));
-      const int tail_st = (K % BKS) ? nstg - 1 : nstg;  // the window stage, if any
+      const int tail_w = (K % BKS) ? nwin - 1 : nwin;  // the re-read window, if any
       for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
         const uint32_t d = tmem + (it & 1) * BN;
         // accumulator it & 1 was last used by item it - 2
@@ -295,8 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait1(&dempty[it & 1], d_phase, abort_flag, status)) break;
           if (it & 1) d_phase ^= 1u;
         }
-        uint64_t xdesc = xdesc0 + static_cast<uint64_t>(s_slot * (X_BYTES >> 4));
-        uint64_t wdesc = wdesc0 + static_cast<uint64_t>(s_slot * (W_SMEM >> 4));
+        uint64_t xdesc = xdesc0 + static_cast<uint64_t>(s_slot * WPS * (X_BYTES >> 4));
+        uint64_t wdesc = wdesc0 + static_cast<uint64_t>(s_slot * WPS * (W_SMEM >> 4));
         uint32_t sfa = t_sf + s_slot * kSlotCols;
         for (int st = 0; st < nstg; ++st) {
           if (!wait1(&full[s_slot], s_phase, abort_flag, status)) {
@@ -305,18 +312,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::tc_fence_after();
           // a descriptor addresses shared memory in 16-byte units: +2 per 32 bytes
-          if (st != tail_st) {
-            tc::mma_mx_ss(d, xdesc, wdesc, IDESC | tc::idesc_sf_ids(0, 0), st > 0 ? 1u : 0u, sfa,
-                          sfa + 4);
-            tc::mma_mx_ss(d, xdesc + 2, wdesc + 2, IDESC | tc::idesc_sf_ids(1, 1), 1u, sfa, sfa + 4);
+#pragma unroll
+          for (int v = 0; v < WPS; ++v) {
+            const int w = st * WPS + v;
+            if (w >= nwin) break;
+            const uint64_t xv = xdesc + v * (X_BYTES >> 4), wv = wdesc + v * (W_SMEM >> 4);
+            const uint32_t sv = sfa + 8 * v;
+            if (w != tail_w) {
+              tc::mma_mx_ss(d, xv, wv, IDESC | tc::idesc_sf_ids(0, 0), w > 0 ? 1u : 0u, sv, sv + 4);
+              tc::mma_mx_ss(d, xv + 2, wv + 2, IDESC | tc::idesc_sf_ids(1, 1), 1u, sv, sv + 4);
+            }
+            tc::mma_mx_ss(d, xv + 4, wv + 4, IDESC | tc::idesc_sf_ids(2, 2),
+                          (w != tail_w || w > 0) ? 1u : 0u, sv, sv + 4);
+            tc::mma_mx_ss(d, xv + 6, wv + 6, IDESC | tc::idesc_sf_ids(3, 3), 1u, sv, sv + 4);
           }
-          tc::mma_mx_ss(d, xdesc + 4, wdesc + 4, IDESC | tc::idesc_sf_ids(2, 2),
-                        (st != tail_st || st > 0) ? 1u : 0u, sfa, sfa + 4);
-          tc::mma_mx_ss(d, xdesc + 6, wdesc + 6, IDESC | tc::idesc_sf_ids(3, 3), 1u, sfa, sfa + 4);
           tc::mma_commit(&empty[s_slot]);
           any = true;
-          xdesc += X_BYTES >> 4;
-          wdesc += W_SMEM >> 4;
+          xdesc += WPS * (X_BYTES >> 4);
+          wdesc += WPS * (W_SMEM >> 4);
           sfa += kSlotCols;
           if (++s_slot == NS) {
             s_slot = 0;
@@ -378,25 +391,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::tc_fence_after();
         }
-        const int kb0 = stage_k0(st, K) / 32;
-        // token-scale column c of lane l holds piece row 32c + l
-        const uint32_t* sx = xwords + st * XR;
-        uint32_t wx[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) wx[c] = (32 * c + lane < XR) ? sx[32 * c + lane] : 0x7F7F7F7Fu;
-        uint32_t ww[4];
+        for (int v = 0; v < WPS; ++v) {
+          const int w = st * WPS + v;
+          if (w >= nwin) break;
+          const int kb0 = stage_k0(w, K) / 32;
+          // token-scale column c of lane l holds piece row 32c + l
+          const uint32_t* sx = xwords + w * XR;
+          uint32_t wx[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (live[c]) {
-            const uint16_t* p = reinterpret_cast<const uint16_t*>(wsc[c] + kb0);
-            ww[c] = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 16);
-          } else {
-            ww[c] = 0x7F7F7F7Fu;
+          for (int c = 0; c < 4; ++c) wx[c] = (32 * c + lane < XR) ? sx[32 * c + lane] : 0x7F7F7F7Fu;
+          uint32_t ww[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (live[c]) {
+              const uint16_t* p = reinterpret_cast<const uint16_t*>(wsc[c] + kb0);
+              ww[c] = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 16);
+            } else {
+              ww[c] = 0x7F7F7F7Fu;
+            }
           }
+          const uint32_t col = t_sf + s_slot * kSlotCols + 8 * v;
+          tc::tmem_st4(lane_base + col, wx);
+          tc::tmem_st4(lane_base + col + 4, ww);
         }
-        const uint32_t col = t_sf + s_slot * kSlotCols;
-        tc::tmem_st4(lane_base + col, wx);
-        tc::tmem_st4(lane_base + col + 4, ww);
         tc::tmem_st_wait();
         tc::tc_fence_before();
         __syncwarp();
