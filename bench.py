@@ -59,8 +59,8 @@ def launches_per_layer(T: int, E: int, k: int) -> int:
 # dram bytes (read + write) of one moe_expert_mlp call on the default workload,
 # from an ncu capture of the kernels whose source hashes to TRAFFIC_SRC_SHA;
 # reported only while the source is unchanged
-TRAFFIC_BYTES = 438084864  # gate/up 285.20 + 4.69 MB, down 144.20 + 4.00 MB (read + write)
-TRAFFIC_SRC_SHA = "05c0ddecd2ddd184"
+TRAFFIC_BYTES = 438201856  # gate/up 285.19 + 4.95 MB, down 144.21 + 3.86 MB (read + write)
+TRAFFIC_SRC_SHA = "9a527ef1e275f912"
 TRAFFIC_WORKLOAD = DEFAULT_WORKLOAD
 
 
@@ -398,6 +398,30 @@ def run_ours(args):
     t_roof_meas = max(layer_bytes / (hbm * 1e9), layer_flops / (tc_sust * 1e12))
     t_roof_spec = max(layer_bytes / 8e12, layer_flops / 2.25e15)
 
+    # ---- router scores fused with the top-k (moe_router_topk) on the same
+    #      tokens, against a seeded bf16 router matrix [E][D]
+    router = None
+    if D % 64 == 0:
+        w_router = torch.from_numpy(syn.normal_bf16(wl.seed, 40, (E, D), sigma=1.0 / D ** 0.5)
+                                    .view(np.int16)).to(dev).view(torch.bfloat16)
+        r_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        r_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        r_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        r_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps + 2):
+            flush.fill_(i & 0xFF)
+            if i >= 2:
+                r_starts[i - 2].record(stream)
+            moe.moe_router_topk(x, w_router, k, r_idx, r_w, None, None, stream)
+            if i >= 2:
+                r_ends[i - 2].record(stream)
+        torch.cuda.synchronize()
+        r_ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in zip(r_starts, r_ends))
+        r_bytes = T * D * 2 + E * D * 2 + T * k * 8
+        router = {"call": "moe_router_topk", "ms": r_ms, "bytes": r_bytes,
+                  "GB/s": r_bytes / (r_ms / 1e3) / 1e9,
+                  "TFLOP/s": 2.0 * T * D * E / (r_ms / 1e3) / 1e12}
+
     # ---- end to end through the C ABI with host buffers
     x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     lg_host = torch.from_numpy(lg_np).pin_memory()
@@ -445,6 +469,7 @@ def run_ours(args):
                            "frac_of_measured": t_roof_meas / (ms_per_step / 1e3),
                            "frac_of_spec_8TBs_2.25PF": t_roof_spec / (ms_per_step / 1e3),
                            "touched_experts": touched},
+        "router": router,
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": launches_per_layer(T, E, k) * args.steps,
         "wall_s_timed_region": wall, "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),

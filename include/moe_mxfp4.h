@@ -140,6 +140,26 @@ MOE_API moe_status mxfp4_quantize(const uint16_t* w_bf16, int64_t rows, int64_t 
 MOE_API moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
                      int32_t* topk_idx, float* topk_w, moe_stream stream);
 
+/* moe_router_topk -- router scores fused with moe_route.
+ * Passage: "Welcome GPT OSS ..." (summary), section 4 (token-choice MoE, a
+ * router scoring every token against every expert, softmax-after-topk);
+ * aitrends.kr talk summary (4 active experts).
+ * logits[t][e] = sum_d x[t][d] * w_router[e][d]: bf16 inputs, exact
+ * products, fp32 accumulation on the tensor core (order unspecified); then
+ * topk_idx / topk_w exactly as moe_route computes them from those logits.
+ *   x        in   [T][D] bf16, D a multiple of 64 in [64, 16384]
+ *   w_router in   [E][D] bf16 (one row per expert), E <= 256
+ *   logits   out  nullable; [T][E] fp32 when given
+ *   topk_idx out  [T][k] int32; topk_w out [T][k] fp32
+ *   d_status out  nullable; MOE_ERR_TIMEOUT if a bounded wait gave up
+ *                 (never written otherwise)
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA.                                                          */
+MOE_API moe_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T,
+                                   int32_t D, int32_t E, int32_t k, float* logits,
+                                   int32_t* topk_idx, float* topk_w, int32_t* d_status,
+                                   moe_stream stream);
+
 /* moe_permute -- group the T*k routed slots by expert.
  * Passage: "MXFP4-based MoE technical review", section 4 (routing and its
  * parallelisation as the core difficulty of sparse experts).

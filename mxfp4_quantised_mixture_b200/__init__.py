@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
     lib.mxfp4_quantize.restype = st
     lib.moe_route.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     lib.moe_route.restype = st
+    lib.moe_router_topk.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.moe_router_topk.restype = st
     lib.moe_permute.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_permute.restype = st
     lib.moe_expert_mlp.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -125,6 +127,17 @@ def moe_route(logits, k: int, topk_idx, topk_w, stream=None) -> None:
     _check("moe_route", lib.moe_route(_p(logits), T, E, k, _p(topk_idx), _p(topk_w), _s(stream)))
 
 
+def moe_router_topk(x, w_router, k: int, topk_idx, topk_w, logits=None, d_status=None,
+                    stream=None) -> None:
+    """x [T][D] bf16, w_router [E][D] bf16 -> topk_idx [T][k] i32, topk_w [T][k] f32
+    (and logits [T][E] f32 when given)."""
+    T, D = x.shape
+    E = w_router.shape[0]
+    _check("moe_router_topk", lib.moe_router_topk(_p(x), _p(w_router), T, D, E, k, _p(logits),
+                                                  _p(topk_idx), _p(topk_w), _p(d_status),
+                                                  _s(stream)))
+
+
 def moe_permute(topk_idx, x, shape: moe_shape, counts, offsets, sorted_slot, slot_pos, x_perm,
                 ws=None, stream=None) -> None:
     _check("moe_permute", lib.moe_permute(_p(topk_idx), _p(x), shape, _p(counts), _p(offsets),
@@ -171,7 +184,8 @@ def alloc_workspace(shape: moe_shape, which: int, device="cuda"):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-__all__ = ["moe_shape", "make_shape", "MoeError", "mxfp4_quantize", "moe_route", "moe_permute",
+__all__ = ["moe_shape", "make_shape", "MoeError", "mxfp4_quantize", "moe_route",
+           "moe_router_topk", "moe_permute",
            "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_layer_forward_static",
            "moe_workspace_size",
            "moe_status_string", "alloc_workspace", "lib", "LIB_PATH"]

@@ -87,6 +87,12 @@ moe_status route_launch(const float* logits, int T, int E, int k, int32_t* idx, 
 
 }  // namespace moe
 
+namespace moe {
+moe_status router_launch(const uint16_t* x, const uint16_t* w_router, int T, int D, int E, int k,
+                         float* logits, int32_t* idx, float* wts, int32_t* status,
+                         cudaStream_t stream);
+}  // namespace moe
+
 extern "C" moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
                                 int32_t* topk_idx, float* topk_w, moe_stream stream) {
   using namespace moe;

@@ -1,0 +1,282 @@
+// Router: logits = x . W_router^T fused with token-choice top-k and the
+// softmax over the chosen experts.
+//
+// "Welcome GPT OSS, the new open-source model family from OpenAI" (summary),
+// section 4: token-choice MoE with the softmax taken after the top-k;
+// aitrends.kr talk summary, "Architecture details": 4 of 32 or 128 experts.
+// The router scores every token against every expert; the routing that
+// follows is the one moe_route computes from given logits.
+//
+// One CTA per 128 tokens.  The scores are a bf16 GEMM on the tensor core:
+// tokens on the MMA's M side (128), the experts on N (E padded to a multiple
+// of 16, at most 256), K = D in stages of 64 (one 128-byte swizzle row of
+// bf16), both operands by TMA into shared memory, the fp32 accumulator in
+// tensor memory.  Four epilogue warps give each token row to one thread,
+// which reads its E scores from tensor memory, keeps a running top-8 list in
+// registers (value descending, index ascending), and applies the softmax
+// over the first k in fp32 with the same summation order as moe_route, so
+// the routing equals moe_route applied to the returned logits.
+// Every wait is bounded (2 s); on expiry the kernel records MOE_ERR_TIMEOUT
+// in the status word and returns after draining its copies and MMAs.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "tc_sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BKR = 64;                 // K elements per stage (128 bytes of bf16)
+constexpr int MT = 128;                 // tokens per CTA (MMA M)
+constexpr int A_BYTES = MT * BKR * 2;   // token rows per stage
+constexpr int NSR = 4;                  // stages in the ring
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__host__ __device__ inline int smem_bytes_router(int npad) {
+  return 1024 + NSR * (A_BYTES + npad * BKR * 2) + 256;
+}
+
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    router_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                  int T, int D, int E, int npad, int k, float* __restrict__ logits,
+                  int32_t* __restrict__ idx, float* __restrict__ wts, int32_t* __restrict__ status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int b_bytes = npad * BKR * 2;
+  uint8_t* as = smem;
+  uint8_t* bs = smem + NSR * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bs + NSR * b_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = full + NSR;
+  uint64_t* dfull = empty + NSR;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(dfull + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nstg = D / BKR;
+  const int t0 = blockIdx.x * MT;
+  int tcols = 32;
+  while (tcols < npad) tcols *= 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSR; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(dfull, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+    tc::tma_prefetch_desc(&map_x);
+    tc::tma_prefetch_desc(&map_w);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_holder, tcols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int st = 0; st < nstg; ++st) {
+        const int s = st % NSR, u = st / NSR;
+        if (u > 0 && !tc::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitLimitNs)) {
+          *abort_flag = 1;
+          record_status(status, MOE_ERR_TIMEOUT);
+          break;
+        }
+        tc::mbar_arrive_expect_tx(&full[s], A_BYTES + b_bytes);
+        tc::tma_load_2d(as + s * A_BYTES, &map_x, &full[s], st * BKR, t0);
+        tc::tma_load_2d(bs + s * b_bytes, &map_w, &full[s], st * BKR, 0);
+        ++issued;
+      }
+      for (int st = max(0, issued - NSR); st < issued; ++st)
+        tc::mbar_wait(&full[st % NSR], (st / NSR) & 1, abort_flag, kWaitLimitNs / 8);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(MT, npad);
+      int done = 0;
+      for (int st = 0; st < nstg; ++st) {
+        const int s = st % NSR;
+        if (!tc::mbar_wait(&full[s], (st / NSR) & 1, abort_flag, kWaitLimitNs)) {
+          *abort_flag = 1;
+          record_status(status, MOE_ERR_TIMEOUT);
+          break;
+        }
+        tc::tc_fence_after();
+        const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(as + s * A_BYTES));
+        const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(bs + s * b_bytes));
+        // a descriptor addresses shared memory in 16-byte units: +2 per 16 bf16
+#pragma unroll
+        for (int kk = 0; kk < BKR / 16; ++kk)
+          tc::mma_bf16_ss(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (st | kk) != 0);
+        tc::mma_commit(&empty[s]);
+        ++done;
+      }
+      if (done > 0)
+        tc::mma_commit(dfull);
+      else
+        tc::mbar_arrive(dfull);
+    }
+  } else {
+    const int q = warp & 3;
+    const int m = q * 32 + lane;
+    const int t = t0 + m;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    bool ok = tc::mbar_wait(dfull, 0, abort_flag, kWaitLimitNs);
+    ok = __all_sync(0xFFFFFFFFu, ok) && *abort_flag == 0;
+    if (ok) {
+      tc::tc_fence_after();
+      float tv[8];
+      int ti[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        tv[j] = -INFINITY;
+        ti[j] = 0x7FFFFFFF;
+      }
+      for (int c = 0; c < npad; c += 16) {
+        uint32_t r[16];
+        tc::tmem_ld16(tmem + lane_base + c, r);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = c + i;
+          if (e >= E) break;
+          const float v = __uint_as_float(r[i]);
+          if (logits && t < T) logits[static_cast<int64_t>(t) * E + e] = v;
+          // experts arrive in index order: an equal value never displaces an
+          // earlier one, so ties keep the lower index
+          if (better(v, e, tv[7], ti[7])) {
+            tv[7] = v;
+            ti[7] = e;
+#pragma unroll
+            for (int j = 7; j > 0; --j) {
+              if (better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
+                const float fv = tv[j];
+                tv[j] = tv[j - 1];
+                tv[j - 1] = fv;
+                const int fi = ti[j];
+                ti[j] = ti[j - 1];
+                ti[j - 1] = fi;
+              }
+            }
+          }
+        }
+      }
+      if (t < T) {
+        // softmax over the first k, summed in the order of moe_route's
+        // butterfly over lanes j = 0..7 (zero beyond k)
+        float ex[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ex[j] = j < k ? expf(tv[j] - tv[0]) : 0.f;
+        const float z = ((ex[0] + ex[4]) + (ex[2] + ex[6])) + ((ex[1] + ex[5]) + (ex[3] + ex[7]));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < k) {
+            idx[static_cast<int64_t>(t) * k + j] = ti[j];
+            wts[static_cast<int64_t>(t) * k + j] = ex[j] / z;
+          }
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::mbar_wait(dfull, 0, abort_flag, kWaitLimitNs / 8);
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, tcols);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return static_cast<EncodeTiledFn>(nullptr);
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// bf16 rows [rows][K], box = 64 K x box_rows rows, 128-byte swizzle
+bool make_rows_map(CUtensorMap* map, const uint16_t* base, int64_t rows, int K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {BKR, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+moe_status router_launch(const uint16_t* x, const uint16_t* w_router, int T, int D, int E, int k,
+                         float* logits, int32_t* idx, float* wts, int32_t* status,
+                         cudaStream_t stream) {
+  if (T == 0) return MOE_OK;
+  const int npad = (E + 15) / 16 * 16;
+  CUtensorMap mx, mw;
+  if (!make_rows_map(&mx, x, T, D, MT) || !make_rows_map(&mw, w_router, E, D, npad))
+    return MOE_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes_router(256)) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    attr_done = true;
+  }
+  const int grid = (T + MT - 1) / MT;
+  router_kernel<<<grid, kThreads, smem_bytes_router(npad), stream>>>(mx, mw, T, D, E, npad, k,
+                                                                     logits, idx, wts, status);
+  return launch_status();
+}
+
+}  // namespace moe
+
+extern "C" moe_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T,
+                                      int32_t D, int32_t E, int32_t k, float* logits,
+                                      int32_t* topk_idx, float* topk_w, int32_t* d_status,
+                                      moe_stream stream) {
+  using namespace moe;
+  if (T < 0 || T > (1 << 20) || E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MOE_ERR_SHAPE;
+  if (D < 64 || D > 16384 || (D % 64) != 0) return MOE_ERR_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_router, topk_idx, topk_w};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (logits && !aligned16(logits)) return MOE_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_device();
+  if (st != MOE_OK) return st;
+  return router_launch(x, w_router, T, D, E, k, logits, topk_idx, topk_w, d_status,
+                       static_cast<cudaStream_t>(stream));
+}

@@ -55,6 +55,7 @@ def _L():
         lib.oracle_mxfp4_quantize_mt.restype = i64
         lib.oracle_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp]
         lib.oracle_route.argtypes = [vp, i64, i32, i32, vp, vp]
+        lib.oracle_router_logits.argtypes = [vp, vp, i64, i32, i32, vp]
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
         lib.oracle_gather.argtypes = [vp, vp, i64, i32, i32, vp]
         lib.oracle_expert_mlp.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32]
@@ -128,6 +129,19 @@ def route(logits: np.ndarray, k: int) -> tuple[np.ndarray, np.ndarray]:
     w = np.empty((T, k), dtype=np.float64)
     _L().oracle_route(_p(lg), T, E, k, _p(idx), _p(w))
     return idx, w
+
+
+def router_logits(x_bf16: np.ndarray, w_bf16: np.ndarray) -> np.ndarray:
+    """x [T][D] and w [E][D] as bf16 bit patterns (uint16) -> fp64 [T][E]
+    scores x . w^T (the router before routing)."""
+    x = _c(x_bf16, np.uint16)
+    w = _c(w_bf16, np.uint16)
+    T, D = x.shape
+    E = w.shape[0]
+    assert w.shape[1] == D
+    out = np.empty((T, E), dtype=np.float64)
+    _L().oracle_router_logits(_p(x), _p(w), T, D, E, _p(out))
+    return out
 
 
 def permute(idx: np.ndarray, E: int):

@@ -235,6 +235,19 @@ void oracle_route(const float* logits, int64_t T, int E, int k, int32_t* idx, do
   }
 }
 
+/* router scores [P2 s4: a router scores every token against every expert]:
+ * logits[t][e] = sum_d x[t][d] * w[e][d] over bf16 inputs, in fp64, d ascending */
+void oracle_router_logits(const uint16_t* x, const uint16_t* w, int64_t T, int D, int E,
+                          double* logits) {
+  for (int64_t t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d)
+        acc += oracle_bf16_value(x[t * D + d]) * oracle_bf16_value(w[(int64_t)e * D + d]);
+      logits[t * E + e] = acc;
+    }
+}
+
 /* group slots by expert: counting sort, ascending slot order within expert */
 void oracle_permute(const int32_t* idx, int64_t T, int E, int k, int32_t* counts,
                     int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos) {

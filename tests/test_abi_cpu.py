@@ -102,3 +102,17 @@ def test_bad_arguments_rejected_before_the_device():
     assert L.moe_expert_mlp(16, 16, sh, 32, 16, 32, 16, 16, 16, 16, mlp - 1, None) == moe.MOE_ERR_WORKSPACE
     assert L.moe_combine(16, 16, 16, sh, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_permute(16, 16, sh, None, 16, 16, 16, 16, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_router_arguments_rejected_before_the_device():
+    L = moe.lib
+    # (x, w_router, T, D, E, k, logits, idx, w, d_status, stream)
+    assert L.moe_router_topk(16, 16, 4, 96, 8, 4, None, 16, 16, None, None) == moe.MOE_ERR_SHAPE
+    assert L.moe_router_topk(16, 16, 4, 32, 8, 4, None, 16, 16, None, None) == moe.MOE_ERR_SHAPE
+    assert L.moe_router_topk(16, 16, 4, 128, 0, 1, None, 16, 16, None, None) == moe.MOE_ERR_SHAPE
+    assert L.moe_router_topk(16, 16, 4, 128, 300, 4, None, 16, 16, None, None) == moe.MOE_ERR_SHAPE
+    assert L.moe_router_topk(16, 16, 4, 128, 4, 5, None, 16, 16, None, None) == moe.MOE_ERR_SHAPE
+    assert L.moe_router_topk(16, 16, 0, 128, 8, 4, None, 16, 16, None, None) == moe.MOE_OK
+    assert L.moe_router_topk(None, 16, 4, 128, 8, 4, None, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_router_topk(16, 24, 4, 128, 8, 4, None, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_router_topk(16, 16, 4, 128, 8, 4, 40, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG

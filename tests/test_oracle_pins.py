@@ -464,3 +464,54 @@ def test_golden_digest_of_tiny_workload():
         "out": hashlib.sha256(out.tobytes()).hexdigest(),
     }
     assert got == want
+
+
+# ------------------------------------------------------------------- router
+# "Welcome GPT OSS ..." (summary), section 4: a router scores every token
+# against every expert; the scores are a plain dot product of the token's
+# activations with the expert's router row.
+
+
+def _bits_value(b: int) -> Fraction:
+    """Exact rational value of a finite bf16 bit pattern, decoded from its
+    fields (sign, 8-bit exponent, 7-bit mantissa) without the oracle."""
+    sign = -1 if b & 0x8000 else 1
+    e = (b >> 7) & 0xFF
+    m = b & 0x7F
+    if e == 0:
+        return sign * Fraction(m, 128) * Fraction(2) ** -126
+    return sign * (1 + Fraction(m, 128)) * Fraction(2) ** (e - 127)
+
+
+def test_router_one_hot_rows_select_activations():
+    # a router row with a single 1.0 at column d(e) scores x[t][d(e)] exactly
+    T, D, E = 5, 64, 7
+    x = syn.normal_bf16(21, 900, (T, D))
+    w = np.zeros((E, D), np.uint16)
+    cols = [3, 0, 63, 17, 17, 40, 9]
+    for e, d in enumerate(cols):
+        w[e, d] = 0x3F80  # 1.0
+    got = oracle.router_logits(x, w)
+    want = syn.bf16_bits_to_f32(x[:, cols]).astype(np.float64)
+    assert np.array_equal(got, want)
+
+
+def test_router_matches_exact_rational_sums():
+    # small exponent range: every partial sum is exact in fp64, so the oracle
+    # must equal the exact rational dot product
+    T, D, E = 3, 16, 4
+    x = syn.normal_bf16(22, 901, (T, D))
+    w = syn.normal_bf16(22, 902, (E, D), sigma=0.5)
+    got = oracle.router_logits(x, w)
+    for t in range(T):
+        for e in range(E):
+            exact = sum(_bits_value(int(x[t, d])) * _bits_value(int(w[e, d])) for d in range(D))
+            assert got[t, e] == float(exact)
+
+
+def test_router_row_permutation_permutes_columns():
+    T, D, E = 4, 128, 9
+    x = syn.normal_bf16(23, 903, (T, D))
+    w = syn.normal_bf16(23, 904, (E, D), sigma=0.05)
+    perm = np.array([4, 8, 0, 3, 1, 7, 2, 6, 5])
+    assert np.array_equal(oracle.router_logits(x, w[perm]), oracle.router_logits(x, w)[:, perm])
