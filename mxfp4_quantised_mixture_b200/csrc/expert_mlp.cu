@@ -25,7 +25,7 @@
 // MMA shape: M = 128 token rows (the hi and lo pieces of up to 64 tokens,
 // interleaved: row 2t = hi of token t, row 2t + 1 = lo), N = 128 weight rows,
 // K = 32.  With the weights on N an MMA covers 128 rows x 32 codes and runs at
-// the tensor core's full rate (64 cycles), so a 128-K stage of 8 KB of codes
+// the tensor core's full rate (64 cycles), so a 128-K window of 8 KB of codes
 // costs 256 cycles of MMA, under the ~370 cycles the SM's share of HBM
 // bandwidth needs to deliver it; narrower MMAs are bound by their issue rate.
 // The epilogue adds rows 2t and 2t + 1 (neighbouring lanes).
@@ -34,24 +34,25 @@
 //     a lane holds both halves of SwiGLU; output h [S][F] bf16.
 //   * down: 128 rows of the [D][F] matrix; output y_perm [S][D] bf16.
 // The kernel is persistent: one CTA per SM walks the work items (token tile,
-// weight slice) b, b + grid, ...; its copy ring (up to 12 stages) runs on
+// weight slice) b, b + grid, ...; its copy ring (up to 12 stages of two
+// 128-K windows each, so one barrier round trip covers 256 of K) runs on
 // across items, the weight-scale block of an item is double-buffered and so
 // is the accumulator, so one item's epilogue overlaps the next item's MMAs.
 // Warp roles (14 warps):
 //   warp 0      producer: per item the weight-scale bytes and the token-scale
-//               words (bulk copies), per 128-K stage the weight codes (TMA,
+//               words (bulk copies), per 128-K window the weight codes (TMA,
 //               8 KB of packed codes that land as the 16 KB one-byte-per-code
 //               layout the MMA reads) and the token pieces (TMA, 2 NT x 128 B)
-//   warp 1      tensor-memory owner and MMA issuer: 4 MMAs per stage
-//   warps 2-5   scale writers: per stage they copy the token scales and the
+//   warp 1      tensor-memory owner and MMA issuer: 4 MMAs per window
+//   warps 2-5   scale writers: per window they copy the token scales and the
 //               weight scales (both from the item's auxiliary block) into the
 //               stage slot's scale columns in tensor memory, every lane quarter
 //               its own copy, and add their arrival to the stage's barrier, so
 //               the MMA thread waits on one barrier per stage
 //   warps 6-13  epilogue: two warps per lane quarter, 64 accumulator columns
 //               each; a quarter whose tokens are all padding is skipped
-// When K is not a multiple of 128 the last stage re-reads the window
-// [K - 128, K) and issues only the MMAs over its new 32-element blocks.
+// When K is not a multiple of 128 the last window re-reads [K - 128, K) and
+// issues only the MMAs over its new 32-element blocks.
 // The token pieces sit in a tile-padded layout (tile t owns piece rows
 // [2 t NT, 2 t NT + 2 NT)), so every copy of a tile's rows is aligned and
 // whole; the MMA's 128-row view of a stage narrower than 128 rows reads on
@@ -73,7 +74,7 @@ constexpr int WPS = 2;              // windows per pipeline stage
 constexpr int BN = 128;             // weight rows per work item (MMA N)
 constexpr int MM = 128;             // MMA M: token piece rows
 constexpr int W_SMEM = BN * BKS;    // one byte per code in shared memory
-constexpr int W_TX = BN * BKS / 2;  // bytes the stage's weight copy reads
+constexpr int W_TX = BN * BKS / 2;  // bytes one window's weight copy reads
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (6 + kEpiWarps);
 constexpr int kMaxStages = 12;      // copy ring depth limit (stage slot s also owns scale slot s)
@@ -104,7 +105,8 @@ __host__ __device__ inline SmemLayout smem_layout(int NT, int NS, int NB, int K)
   return L;
 }
 
-// first K element of stage st
+// first K element of 128-K window st; the last window of a K that is not a
+// multiple of 128 is moved back to end at K
 __host__ __device__ __forceinline__ int stage_k0(int st, int K) {
   return st * BKS < K - BKS ? st * BKS : K - BKS;
 }
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const Tile* __restrict__ tiles, const int* __restrict__ n_tiles_dev,
                     int rows_per_expert, int K, int NS, int NB, int out_ld,
                     uint16_t* __restrict__ out, int32_t* __restrict__ status) {
-  constexpr int XR = 2 * NT;  // token piece rows per stage
+  constexpr int XR = 2 * NT;  // token piece rows per window
   constexpr uint32_t X_BYTES = XR * BKS;
   constexpr uint32_t IDESC = tc::idesc_mx(tc::kFmtE4M3, tc::kFmtE2M1, MM, BN);
   static_assert(XR <= MM && (X_BYTES % 1024) == 0, "token tile of 8..64 tokens");
@@ -542,11 +544,11 @@ __global__ void plan_tiles_kernel(const int32_t* __restrict__ offsets, int E, in
 
 // Exact two-piece E4M3 split of bf16 rows (see the file comment), written in
 // the tile-padded layout: piece rows [2 * tiles * NT][K] bytes, row 2p = hi
-// and 2p + 1 = lo of padded row p = t NT + i, and, per tile and stage, the
-// scale words [2 NT] in the same row order (byte b of a word = E8M0 scale of
-// the stage's 32-element block b).  One warp per (padded row, stage); lane l
-// holds elements 4l..4l+3 of the stage's 128-element window, a block is 8
-// lanes.  Padded rows get zero pieces.
+// and 2p + 1 = lo of padded row p = t NT + i, and, per tile and 128-K window,
+// the scale words [2 NT] in the same row order (byte b of a word = E8M0 scale
+// of the window's 32-element block b).  One warp per (padded row, window);
+// lane l holds elements 4l..4l+3 of the window, a block is 8 lanes.  Padded
+// rows get zero pieces.
 __global__ void __launch_bounds__(256) split_rows_kernel(
     const uint16_t* __restrict__ src, int K, const Tile* __restrict__ tiles,
     const int* __restrict__ n_tiles, int NT, int64_t padded_rows, uint8_t* __restrict__ pieces,
@@ -590,7 +592,7 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
     hi4 |= static_cast<uint32_t>(h8) << (8 * j);
     lo4 |= static_cast<uint32_t>(l8) << (8 * j);
   }
-  // the window stage re-reads [K - 128, 128 st): only its new elements are written
+  // a moved-back last window re-reads [K - 128, 128 st): only its new elements are written
   if (k >= st * BKS) {
     *reinterpret_cast<uint32_t*>(pieces + (2 * p) * K + k) = hi4;
     *reinterpret_cast<uint32_t*>(pieces + (2 * p + 1) * K + k) = lo4;
@@ -694,7 +696,7 @@ constexpr int kMaxSmemPerCta = 227 * 1024;
 int smem_bytes(int NT, int NS, int NB, int K) { return smem_layout(NT, NS, NB, K).total + 1024; }
 
 // token-tile width: about twice the mean rows per expert, 16..64; then the
-// deepest copy ring (up to 8 stages) beside a double-buffered weight-scale
+// deepest copy ring (up to 12 stages) beside a double-buffered weight-scale
 // block, with at least 4 stages; failing that, a single scale block
 GemmConfig choose_config(const moe_shape& sh) {
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
