@@ -10,7 +10,10 @@ them are pinned by ``tests/test_oracle_pins.py`` to facts fixed by the pages
 and by mathematics (exhaustive decode table, brute-force encoding,
 hand-derived blocks, brute-force top-k, permutation invariants, a dense
 per-token restatement, and the single-expert case against fp64
-``torch.matmul``); no function is "parity unpinned".
+``torch.matmul``), and the training-style quantiser by
+``tests/test_oracle_sr_rht_pins.py`` (Philox known answers,
+``scipy.linalg.hadamard``, exact counts over all uniforms); no function is
+"parity unpinned".
 """
 from __future__ import annotations
 
@@ -54,6 +57,15 @@ def _L():
         lib.oracle_mxfp4_quantize_mt.argtypes = [vp, i64, i64, vp, vp, i32]
         lib.oracle_mxfp4_quantize_mt.restype = i64
         lib.oracle_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp]
+        u32, u64 = ctypes.c_uint32, ctypes.c_uint64
+        lib.oracle_philox4x32_10.argtypes = [vp, vp, vp]
+        lib.oracle_sr_uniform16.argtypes = [u64, u64]
+        lib.oracle_sr_uniform16.restype = u32
+        lib.oracle_rht32.argtypes = [vp, u32, vp]
+        lib.oracle_sr_code.argtypes = [dbl, u32]
+        lib.oracle_sr_code.restype = ctypes.c_uint8
+        lib.oracle_mxfp4_quantize_sr_rht.argtypes = [vp, i64, i64, u32, vp, u64, vp, vp, i32]
+        lib.oracle_mxfp4_quantize_sr_rht.restype = i64
         lib.oracle_route.argtypes = [vp, i64, i32, i32, vp, vp]
         lib.oracle_router_logits.argtypes = [vp, vp, i64, i32, i32, vp]
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
@@ -107,6 +119,60 @@ def mxfp4_quantize(w_bf16: np.ndarray) -> tuple[np.ndarray, np.ndarray, int]:
     q = np.empty(w.shape[:-1] + (K // 2,), dtype=np.uint8)
     s = np.empty(w.shape[:-1] + (K // 32,), dtype=np.uint8)
     bad = _L().oracle_mxfp4_quantize_mt(_p(w), rows, K, _p(q), _p(s), _threads())
+    return q, s, int(bad)
+
+
+# flags of the training-style quantiser ("MXFP4-based MoE technical review",
+# sections 2 and 4): a random-sign Hadamard transform of each 32-block along K,
+# and stochastic rounding
+QUANT_RHT = 1
+QUANT_SR = 2
+
+
+def philox4x32_10(ctr, key) -> tuple[int, int, int, int]:
+    """Philox4x32-10 (Salmon et al., SC 2011) of a 4-word counter and 2-word key."""
+    c = np.asarray(ctr, dtype=np.uint32).copy()
+    k = np.asarray(key, dtype=np.uint32).copy()
+    out = np.zeros(4, dtype=np.uint32)
+    _L().oracle_philox4x32_10(_p(c), _p(k), _p(out))
+    return tuple(int(v) for v in out)
+
+
+def sr_uniform16(seed: int, n: int) -> int:
+    """16-bit uniform that element n of a call keyed by ``seed`` draws."""
+    return int(_L().oracle_sr_uniform16(int(seed), int(n)))
+
+
+def rht32(x: np.ndarray, sign_word: int) -> np.ndarray:
+    """y = H (s . x) of one 32-element block (unnormalised Sylvester H)."""
+    xv = _c(x, np.float64)
+    assert xv.shape == (32,)
+    y = np.empty(32, dtype=np.float64)
+    _L().oracle_rht32(_p(xv), int(sign_word) & 0xFFFFFFFF, _p(y))
+    return y
+
+
+def sr_code(v: float, u: int) -> int:
+    """Stochastic rounding of v >= 0 onto the E2M1 magnitudes, 16-bit uniform u."""
+    return int(_L().oracle_sr_code(float(v), int(u)))
+
+
+def mxfp4_quantize_sr_rht(w_bf16: np.ndarray, flags: int, signs: np.ndarray | None,
+                          seed: int) -> tuple[np.ndarray, np.ndarray, int]:
+    """bf16 bits [..., K] -> (codes, scales, #non-finite blocks) with the
+    optional transform (``signs`` [K/32] uint32) and stochastic rounding."""
+    w = _c(w_bf16, np.uint16)
+    K = w.shape[-1]
+    rows = w.size // K if K else 0
+    q = np.empty(w.shape[:-1] + (K // 2,), dtype=np.uint8)
+    s = np.empty(w.shape[:-1] + (K // 32,), dtype=np.uint8)
+    if signs is None:
+        sg = np.zeros(max(1, K // 32), dtype=np.uint32)
+    else:
+        sg = _c(signs, np.uint32)
+        assert sg.shape == (K // 32,)
+    bad = _L().oracle_mxfp4_quantize_sr_rht(_p(w), rows, K, int(flags), _p(sg), int(seed), _p(q),
+                                            _p(s), _threads())
     return q, s, int(bad)
 
 

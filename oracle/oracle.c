@@ -210,6 +210,206 @@ void oracle_mxfp4_decode(const uint8_t* q, const uint8_t* s, int64_t rows, int64
     }
 }
 
+/* ------------------------------------- training-style quantiser [P4 s2, s4] */
+/*
+ * "MXFP4-based MoE technical review", sections 2 and 4: MXFP4 training keeps
+ * its quality with stochastic rounding and a random Hadamard transform.  The
+ * page names the two techniques and no more; the readings taken here are:
+ *  - the transform acts on each 32-element block along K (the block that
+ *    shares one scale): y = H (s . x), H the 32 x 32 Sylvester Hadamard
+ *    matrix (+1/-1 entries, H[i][j] = (-1)^popcount(i & j)), unnormalised,
+ *    s a random sign per position j of block column K/32 given by the caller
+ *    (bit j of signs[block column] set = negate); (H diag(s)) times its
+ *    transpose is 32 I, so a product of two operands that carry the same
+ *    transform along K is 32 times the plain product;
+ *  - y is the exact value of that sum (fp64 here; every test input keeps it
+ *    exact: 32 bf16 terms whose exponents span far less than 40 binades);
+ *  - stochastic rounding moves |y| / scale to one of its two neighbours on
+ *    the E2M1 grid, the upper one with probability equal to the distance from
+ *    the lower one over the gap, drawn as u < frac with u a 16-bit uniform;
+ *    to keep it unbiased no element may clip, so with rounding stochastic the
+ *    scale exponent is the smallest that brings amax to at most 6:
+ *    byte = 127 + ceil(log2(amax / 6)), clamped to [0, 254];
+ *  - uniforms: Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+ *    numbers: as easy as 1, 2, 3", SC 2011) keyed by the 64-bit seed; element
+ *    n = r K + c of the call draws from the counter (n / 8 low word, n / 8
+ *    high word, 0, 0), output word (n % 8) / 2, low half for even n;
+ *  - a transformed element's sign bit is set only for y < 0 (an exact zero
+ *    is code 0); without the transform the sign bit is that of x, as in the
+ *    deterministic quantiser, which this one equals when no flag is set.
+ */
+#define ORACLE_QUANT_RHT 1u
+#define ORACLE_QUANT_SR 2u
+
+/* Philox4x32-10: ten rounds of the two 32 x 32 -> 64-bit products and the
+ * word permutation, the key bumped by the two Weyl constants between rounds */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+  uint32_t k0 = key[0], k1 = key[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+    uint32_t n1 = (uint32_t)p1;
+    uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+    uint32_t n3 = (uint32_t)p0;
+    c0 = n0;
+    c1 = n1;
+    c2 = n2;
+    c3 = n3;
+  }
+  out[0] = c0;
+  out[1] = c1;
+  out[2] = c2;
+  out[3] = c3;
+}
+
+/* the 16-bit uniform of element n of a call keyed by seed */
+uint32_t oracle_sr_uniform16(uint64_t seed, uint64_t n) {
+  uint32_t ctr[4] = {(uint32_t)(n / 8), (uint32_t)((n / 8) >> 32), 0u, 0u};
+  uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t out[4];
+  oracle_philox4x32_10(ctr, key, out);
+  uint32_t word = out[(n % 8) / 2];
+  return (n & 1) ? (word >> 16) : (word & 0xFFFFu);
+}
+
+/* y = H (s . x) of one 32-element block, summed over j ascending */
+void oracle_rht32(const double* x, uint32_t sign_word, double* y) {
+  for (int i = 0; i < 32; ++i) {
+    double acc = 0.0;
+    for (int j = 0; j < 32; ++j) {
+      double xj = ((sign_word >> j) & 1u) ? -x[j] : x[j];
+      acc += (__builtin_popcount((unsigned)(i & j)) & 1) ? -xj : xj;
+    }
+    y[i] = acc;
+  }
+}
+
+/* stochastic rounding of v >= 0 onto the E2M1 magnitudes with the 16-bit
+ * uniform u: the lower neighbour, or the upper one when u / 2^16 < frac */
+uint8_t oracle_sr_code(double v, uint32_t u) {
+  if (v >= 6.0) return 7; /* on the top magnitude (or above it, clipped) */
+  int c = 0;
+  while (E2M1_MAGNITUDE[c + 1] <= v) ++c; /* G[c] <= v < G[c + 1] */
+  double frac = (v - E2M1_MAGNITUDE[c]) / (E2M1_MAGNITUDE[c + 1] - E2M1_MAGNITUDE[c]);
+  return (uint8_t)(((double)u / 65536.0 < frac) ? c + 1 : c);
+}
+
+/* scale byte from the block maximum of |y|: floor(log2 amax) - 2 + 127, and
+ * with stochastic rounding one more when amax / 2^(floor(log2 amax) - 2) > 6 */
+static uint8_t scale_byte_of(double amax, int sr) {
+  if (amax == 0.0) return 0;
+  int e;
+  double m = frexp(amax, &e); /* amax = m 2^e, m in [0.5, 1) */
+  int b = (e - 1) - 2 + 127;
+  if (sr && m > 0.75) b += 1; /* significand above 1.5: 4 * 1.5 = 6 */
+  if (b < 0) b = 0;
+  if (b > 254) b = 254;
+  return (uint8_t)b;
+}
+
+static int64_t quantize_ex_rows(const uint16_t* w, int64_t r0, int64_t r1, int64_t K,
+                                uint32_t flags, const uint32_t* signs, uint64_t seed, uint8_t* q,
+                                uint8_t* s) {
+  const int rht = (flags & ORACLE_QUANT_RHT) != 0, sr = (flags & ORACLE_QUANT_SR) != 0;
+  const int64_t nb = K / 32;
+  int64_t bad = 0;
+  for (int64_t r = r0; r < r1; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      const uint16_t* blk = w + r * K + b * 32;
+      double x[32], y[32];
+      int neg[32], nonfinite = 0;
+      for (int i = 0; i < 32; ++i) {
+        if (((blk[i] >> 7) & 0xFF) == 0xFF) nonfinite = 1;
+        x[i] = oracle_bf16_value(blk[i]);
+      }
+      bad += nonfinite;
+      if (rht) {
+        oracle_rht32(x, signs[b], y);
+        for (int i = 0; i < 32; ++i) neg[i] = y[i] < 0.0;
+      } else {
+        for (int i = 0; i < 32; ++i) {
+          y[i] = x[i];
+          neg[i] = signbit(x[i]) != 0;
+        }
+      }
+      double amax = 0.0;
+      for (int i = 0; i < 32; ++i)
+        if (fabs(y[i]) > amax) amax = fabs(y[i]);
+      uint8_t sb = scale_byte_of(amax, sr);
+      s[r * nb + b] = sb;
+      double scale = ldexp(1.0, (int)sb - 127);
+      for (int i = 0; i < 32; i += 2) {
+        uint8_t c[2];
+        for (int h = 0; h < 2; ++h) {
+          double v = fabs(y[i + h]) / scale; /* exact: a power-of-two scale */
+          uint8_t code;
+          if (sr)
+            code = oracle_sr_code(v, oracle_sr_uniform16(seed, (uint64_t)(r * K + b * 32 + i + h)));
+          else
+            code = e2m1_magnitude_code(v);
+          if (neg[i + h]) code |= 8;
+          c[h] = code;
+        }
+        q[r * (K / 2) + (b * 32 + i) / 2] = (uint8_t)(c[0] | (c[1] << 4));
+      }
+    }
+  }
+  return bad;
+}
+
+typedef struct {
+  const uint16_t* w;
+  int64_t r0, r1, K;
+  uint32_t flags;
+  const uint32_t* signs;
+  uint64_t seed;
+  uint8_t *q, *s;
+  int64_t bad;
+} quant_ex_job;
+
+static void* quant_ex_run(void* arg) {
+  quant_ex_job* j = (quant_ex_job*)arg;
+  j->bad = quantize_ex_rows(j->w, j->r0, j->r1, j->K, j->flags, j->signs, j->seed, j->q, j->s);
+  return NULL;
+}
+
+/* bf16 [rows][K] -> codes + scale bytes with the optional transform and
+ * stochastic rounding above; rows split over threads.  Returns the number of
+ * blocks holding a NaN or infinity. */
+int64_t oracle_mxfp4_quantize_sr_rht(const uint16_t* w, int64_t rows, int64_t K, uint32_t flags,
+                                     const uint32_t* signs, uint64_t seed, uint8_t* q, uint8_t* s,
+                                     int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if (rows < 64) nthreads = 1;
+  pthread_t th[256];
+  quant_ex_job jobs[256];
+  int created[256];
+  int64_t chunk = (rows + nthreads - 1) / nthreads;
+  int used = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    quant_ex_job j = {w, t * chunk, (t + 1) * chunk < rows ? (t + 1) * chunk : rows, K, flags,
+                      signs, seed, q, s, 0};
+    jobs[t] = j;
+    if (jobs[t].r0 >= jobs[t].r1) break;
+    created[t] = pthread_create(&th[t], NULL, quant_ex_run, &jobs[t]) == 0;
+    if (!created[t]) quant_ex_run(&jobs[t]);
+    used = t + 1;
+  }
+  int64_t bad = 0;
+  for (int t = 0; t < used; ++t) {
+    if (created[t]) pthread_join(th[t], NULL);
+    bad += jobs[t].bad;
+  }
+  return bad;
+}
+
 /* ------------------------------------------------------------------ routing */
 
 /* token-choice top-k with softmax over the selected logits [P2 s4, P3] */
