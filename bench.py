@@ -271,6 +271,46 @@ def job_throughput(world: int, tokens_per_rank: int, steps: int, max_total_ms: f
 # -------------------------------------------------------------------- ours
 
 
+def quantiser_timings(moe, w, flush, stream, steps, hbm):
+    """Mean CUDA-event time of mxfp4_quantize and of mxfp4_quantize_sr_rht
+    (both flags) over ``w`` [..., K] bf16, L2 flushed before each call.  The
+    algorithmic bytes are 2 read + 17/32 written per element."""
+    import torch
+
+    K = w.shape[-1]
+    rows = w.numel() // K
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=w.device)
+    sc = torch.empty((rows, K // 32), dtype=torch.uint8, device=w.device)
+    signs = torch.from_numpy(np.random.default_rng(7).integers(0, 1 << 32, size=K // 32, dtype=np.uint64)
+                             .astype(np.uint32).view(np.int32)).to(w.device)
+    elems = rows * K
+    nbytes = elems * 2 + elems // 2 + elems // 32
+    flags = moe.MOE_QUANT_RHT | moe.MOE_QUANT_SR
+    calls = {
+        "mxfp4_quantize": lambda i: moe.mxfp4_quantize(w, q, sc, None, stream),
+        "mxfp4_quantize_sr_rht": lambda i: moe.mxfp4_quantize_sr_rht(w, flags, signs, 1000 + i, q,
+                                                                     sc, None, stream),
+    }
+    out = {"rows": rows, "K": K, "algorithmic_bytes": nbytes}
+    for name, call in calls.items():
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps + 2):
+            flush.fill_(i & 0xFF)
+            if i >= 2:
+                st[i - 2].record(stream)
+            call(i)
+            if i >= 2:
+                en[i - 2].record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in zip(st, en))
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"ms": ms, "GB/s": gbs, "frac_of_hbm": gbs / hbm,
+                     "Gelem/s": elems / (ms / 1e3) / 1e9}
+    out["mxfp4_quantize_sr_rht"]["flags"] = "MOE_QUANT_RHT|MOE_QUANT_SR"
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -310,6 +350,8 @@ def run_ours(args):
         dn = torch.from_numpy(syn.w_down(wl, ex).view(np.int16)).to(dev).view(torch.bfloat16)
         moe.mxfp4_quantize(gu, wgu_q[e0:e0 + len(ex)], wgu_s[e0:e0 + len(ex)], status)
         moe.mxfp4_quantize(dn, wdn_q[e0:e0 + len(ex)], wdn_s[e0:e0 + len(ex)], status)
+        if e0 == 0:
+            gu_first = gu  # kept for the quantiser timings below
         del gu, dn
     torch.cuda.synchronize()
     if int(status.item()) != 0:
@@ -429,6 +471,13 @@ def run_ours(args):
                   "GB/s": r_bytes / (r_ms / 1e3) / 1e9,
                   "TFLOP/s": 2.0 * T * D * E / (r_ms / 1e3) / 1e12}
 
+    # ---- the quantisers, timed on their own over the first chunk of gate/up
+    #      weights (bf16 in, larger than L2): the deterministic one that
+    #      produced the layer's weights, and the training-style one with the
+    #      random-sign Hadamard transform and stochastic rounding
+    quant = quantiser_timings(moe, gu_first, flush, stream, args.steps, hbm)
+    del gu_first
+
     # ---- end to end through the C ABI with host buffers
     x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     lg_host = torch.from_numpy(lg_np).pin_memory()
@@ -477,6 +526,7 @@ def run_ours(args):
                            "frac_of_spec_8TBs_2.25PF": t_roof_spec / (ms_per_step / 1e3),
                            "touched_experts": touched},
         "router": router,
+        "quantize": quant,
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": launches_per_layer(T, E, k) * args.steps,
         "wall_s_timed_region": wall, "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),

@@ -125,6 +125,49 @@ MOE_API moe_status mxfp4_quantize(const uint16_t* w_bf16, int64_t rows, int64_t 
                           uint8_t* q_packed, uint8_t* scales,
                           int32_t* d_status, moe_stream stream);
 
+/* mxfp4_quantize_sr_rht -- training-style bf16 -> MXFP4 quantiser.
+ * Passage: "MXFP4-based MoE technical review", sections 2 and 4 (stochastic
+ * rounding and a random Hadamard transform keep MXFP4 training close to
+ * bf16); the format as for mxfp4_quantize.  Per 32-element block of a row:
+ *   MOE_QUANT_RHT  y = H (s . x), H the unnormalised 32-point Sylvester
+ *                  Hadamard matrix (+1/-1, H[i][j] = (-1)^popcount(i & j)),
+ *                  s_j = -1 where bit j of rht_signs[c / 32] is set (c the
+ *                  element's column); y is exact (fp64) whenever the block's
+ *                  nonzero exponents span under 40 binades.  A product of two
+ *                  operands that carry the same transform along K is 32 times
+ *                  the plain product.  Without the flag y = x.
+ *   scale byte     floor(log2 amax|y|) - 2 + 127; with MOE_QUANT_SR the
+ *                  smallest byte with amax / 2^(byte-127) <= 6, i.e. one more
+ *                  when the significand of amax is above 1.5 (no element
+ *                  clips, so the rounding is unbiased); clamped to [0, 254];
+ *                  an all-zero block gets 0.
+ *   codes          v = |y| / scale rounded to nearest even onto
+ *                  {0,.5,1,1.5,2,3,4,6} (saturating at 6), or, with
+ *                  MOE_QUANT_SR, to the upper neighbour when
+ *                  u / 65536 < (v - lo) / (hi - lo), u the 16-bit uniform of
+ *                  element n = r K + c: Philox4x32-10 (Salmon et al., SC 2011)
+ *                  of counter (n / 8 low, n / 8 high, 0, 0) under key (seed
+ *                  low, seed high), output word (n % 8) / 2, low half for even
+ *                  n.  Sign bit: y < 0 with the transform, else the sign bit
+ *                  of x.  flags == 0 gives exactly mxfp4_quantize's bytes.
+ *   w_bf16    in   [rows][K] bf16, 16-byte aligned
+ *   rows, K   in   as for mxfp4_quantize
+ *   flags     in   MOE_QUANT_RHT | MOE_QUANT_SR, any subset
+ *   rht_signs in   [K/32] uint32, 4-byte aligned; required with MOE_QUANT_RHT,
+ *                  else ignored (may be NULL)
+ *   seed      in   Philox key; the same seed and shape give the same bytes
+ *   q_packed  out  [rows][K/2]; scales out [rows][K/32]; both 16-byte aligned
+ *   d_status  out  nullable; MOE_ERR_NONFINITE if a block holds NaN or Inf
+ *                  (its bytes unspecified); never written otherwise.
+ * Errors: MOE_ERR_INVALID_ARG (unknown flag bits, missing signs, null or
+ * misaligned pointer), MOE_ERR_SHAPE, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.  */
+#define MOE_QUANT_RHT 1u
+#define MOE_QUANT_SR 2u
+MOE_API moe_status mxfp4_quantize_sr_rht(const uint16_t* w_bf16, int64_t rows, int64_t K,
+                                         uint32_t flags, const uint32_t* rht_signs,
+                                         uint64_t seed, uint8_t* q_packed, uint8_t* scales,
+                                         int32_t* d_status, moe_stream stream);
+
 /* moe_route -- token-choice top-k with softmax over the chosen k.
  * Passage: "Welcome GPT OSS ..." (summary), section 4 (token-choice MoE,
  * softmax-after-topk); aitrends.kr talk summary (4 active experts).

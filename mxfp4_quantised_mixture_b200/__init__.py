@@ -26,6 +26,9 @@ MOE_ERR_TIMEOUT = 7
 
 WS_PERMUTE, WS_EXPERT_MLP, WS_LAYER = 0, 1, 2
 
+MOE_QUANT_RHT = 1  # random-sign Hadamard transform of each 32-block along K
+MOE_QUANT_SR = 2   # stochastic rounding
+
 
 class MoeError(RuntimeError):
     def __init__(self, fn: str, status: int):
@@ -51,6 +54,9 @@ def _load() -> ctypes.CDLL:
     st = ctypes.c_int
     lib.mxfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp]
     lib.mxfp4_quantize.restype = st
+    lib.mxfp4_quantize_sr_rht.argtypes = [vp, i64, i64, ctypes.c_uint32, vp, ctypes.c_uint64, vp,
+                                          vp, vp, vp]
+    lib.mxfp4_quantize_sr_rht.restype = st
     lib.moe_route.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     lib.moe_route.restype = st
     lib.moe_router_topk.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
@@ -122,6 +128,19 @@ def mxfp4_quantize(w_bf16, q_packed, scales, d_status=None, stream=None) -> None
                                                 _p(d_status), _s(stream)))
 
 
+def mxfp4_quantize_sr_rht(w_bf16, flags: int, rht_signs, seed: int, q_packed, scales,
+                          d_status=None, stream=None) -> None:
+    """w_bf16 [rows][K] bf16 -> q_packed [rows][K/2] u8, scales [rows][K/32] u8,
+    with the optional transform (MOE_QUANT_RHT; rht_signs [K/32] int32/uint32)
+    and stochastic rounding (MOE_QUANT_SR, Philox keyed by ``seed``)."""
+    K = w_bf16.shape[-1]
+    rows = w_bf16.numel() // K if K else 0
+    _check("mxfp4_quantize_sr_rht",
+           lib.mxfp4_quantize_sr_rht(_p(w_bf16), rows, K, int(flags) & 0xFFFFFFFF, _p(rht_signs),
+                                     int(seed) & 0xFFFFFFFFFFFFFFFF, _p(q_packed), _p(scales),
+                                     _p(d_status), _s(stream)))
+
+
 def moe_route(logits, k: int, topk_idx, topk_w, stream=None) -> None:
     T, E = logits.shape
     _check("moe_route", lib.moe_route(_p(logits), T, E, k, _p(topk_idx), _p(topk_w), _s(stream)))
@@ -184,7 +203,8 @@ def alloc_workspace(shape: moe_shape, which: int, device="cuda"):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-__all__ = ["moe_shape", "make_shape", "MoeError", "mxfp4_quantize", "moe_route",
+__all__ = ["moe_shape", "make_shape", "MoeError", "mxfp4_quantize", "mxfp4_quantize_sr_rht",
+           "MOE_QUANT_RHT", "MOE_QUANT_SR", "moe_route",
            "moe_router_topk", "moe_permute",
            "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_layer_forward_static",
            "moe_workspace_size",

@@ -1,0 +1,270 @@
+// Training-style bf16 -> MXFP4 quantiser: optional random-sign Hadamard
+// transform of every 32-element block and optional stochastic rounding.
+//
+// "MXFP4-based MoE technical review", sections 2 and 4, names stochastic
+// rounding and a random Hadamard transform as what keeps MXFP4 training close
+// to bf16.  What this kernel computes, per 32-element block of a row:
+//   * transform (flag MOE_QUANT_RHT): y = H (s . x), H the unnormalised 32-point
+//     Sylvester Hadamard matrix (H[i][j] = (-1)^popcount(i & j)), s the signs
+//     of the block's column given by the caller.  H diag(s) times its
+//     transpose is 32 I, so a GEMM whose two operands carry the same transform
+//     along K returns 32 times the plain product.  y is exact: the butterfly
+//     runs in fp64, where sums of 32 bf16 terms whose exponents span less than
+//     40 binades carry no rounding;
+//   * scale byte: floor(log2 amax) - 2 + 127, as in the deterministic
+//     quantiser, or, with stochastic rounding, the smallest exponent that keeps
+//     amax / scale <= 6 (one more when the significand of amax is above 1.5),
+//     so that no element clips and the rounding stays unbiased; clamped to
+//     [0, 254];
+//   * codes: |y| / scale (exact) rounded to nearest even onto
+//     {0, .5, 1, 1.5, 2, 3, 4, 6}, or (flag MOE_QUANT_SR) to the upper grid
+//     neighbour when u / 2^16 < (v - lo) / (hi - lo), u the element's 16-bit
+//     uniform from Philox4x32-10 (Salmon, Moraes, Dror and Shaw, SC 2011):
+//     element n of the call uses counter (n / 8, 0, 0) under the 64-bit seed,
+//     output word (n % 8) / 2, low half for even n;
+//   * sign bit: y < 0 with the transform (an exact zero is +0), else the sign
+//     bit of x.  With no flag the call is mxfp4_quantize itself.
+//
+// Layout: one thread per 32-element block.  A warp loads 32 consecutive blocks
+// (2 KB) with coalesced 16-byte loads into a padded shared-memory stage (a
+// block's 64 bytes take 80, so the per-thread reads are free of bank
+// conflicts), decodes its own block into 32 doubles, transforms, encodes and
+// writes its 16 code bytes (the warp's 512 are contiguous) and its scale byte.
+// The fp64 butterfly, Philox and the integer encoding make the kernel
+// instruction-bound rather than HBM-bound.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kStageStride = 5;  // uint4 slots per block in the stage (4 + 1 pad)
+
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u, kPhiloxM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhiloxW0 = 0x9E3779B9u, kPhiloxW1 = 0xBB67AE85u;
+
+// Philox4x32-10 of counter c under key (k0, k1)
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = kPhiloxM0 * c.x, hi0 = __umulhi(kPhiloxM0, c.x);
+    const uint32_t lo1 = kPhiloxM1 * c.z, hi1 = __umulhi(kPhiloxM1, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += kPhiloxW0;
+    k1 += kPhiloxW1;
+  }
+  return c;
+}
+
+// exact fp64 value of a bf16 bit pattern (finite patterns; the exponent field
+// 0xFF gives some finite value, its block is reported as non-finite).  A zero
+// or subnormal m 2^-133 is (2^-81 + m 2^-133) - 2^-81, the first term built
+// from its bits, so no conversion instruction is needed.
+__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
+  const uint32_t e = (b >> 7) & 0xFFu, m = b & 0x7Fu;
+  double d;
+  if (e != 0)
+    d = __hiloint2double(static_cast<int>(((e + 896u) << 20) | (m << 13)), 0);
+  else
+    d = __hiloint2double(static_cast<int>(942u << 20), static_cast<int>(m)) - 0x1p-81;
+  return __hiloint2double(__double2hiint(d) | static_cast<int>((b & 0x8000u) << 16),
+                          __double2loint(d));
+}
+
+// E2M1 magnitude code of v = |y| / scale >= 0, from v's fp64 bit fields:
+//   v >= 1:       binade e = 0, 1, 2 holds 2^e, 1.5 2^e: base code 2 + 2e + (top
+//                 mantissa bit), the other 51 mantissa bits are the fraction of
+//                 the gap (2^(e-1)) to the next code; v >= 8 saturates to 7;
+//   v in [.5, 1): base 1 (0.5), the 52 mantissa bits are the fraction of 0.5;
+//   v < .5:       base 0, fraction 2 v.
+template <bool SR>
+__device__ __forceinline__ uint32_t e2m1_code(double v, uint32_t u) {
+  const uint32_t vh = static_cast<uint32_t>(__double2hiint(v));
+  const uint32_t vl = static_cast<uint32_t>(__double2loint(v));
+  const int ev = static_cast<int>(vh >> 20);  // v >= 0: no sign bit
+  uint32_t code;
+  if (ev >= 1023) {
+    const uint32_t base = 2u + 2u * static_cast<uint32_t>(ev - 1023) + ((vh >> 19) & 1u);
+    const uint64_t R = (static_cast<uint64_t>(vh & 0x7FFFFu) << 32) | vl;  // 51 bits
+    bool up;
+    if (SR)
+      up = (static_cast<uint64_t>(u) << 35) < R;
+    else
+      up = R > (1ull << 50) || (R == (1ull << 50) && (base & 1u));
+    code = min(base + (up ? 1u : 0u), 7u);
+  } else if (ev == 1022) {
+    const uint64_t R = (static_cast<uint64_t>(vh & 0xFFFFFu) << 32) | vl;  // 52 bits
+    const bool up = SR ? (static_cast<uint64_t>(u) << 36) < R : R >= (1ull << 51);
+    code = up ? 2u : 1u;
+  } else {
+    const bool up = SR ? static_cast<double>(u) < v * 131072.0 : v > 0.25;
+    code = up ? 1u : 0u;
+  }
+  return code;
+}
+
+template <bool RHT, bool SR>
+__global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
+    const uint4* __restrict__ w, int64_t nblocks, int64_t nbk, int64_t stride_mod,
+    const uint32_t* __restrict__ signs, uint32_t key0, uint32_t key1, uint4* __restrict__ q,
+    uint8_t* __restrict__ s, int32_t* __restrict__ status) {
+  __shared__ uint4 stage[kWarps][32 * kStageStride];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t warp0 = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  int64_t col = (warp0 * 32 + lane) % nbk;  // block column of this lane's block
+  for (int64_t base = warp0 * 32; base < nblocks; base += nwarps * 32) {
+    // coalesced 16-byte loads of the warp's 32 blocks into the stage
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int p = lane + 32 * j;  // piece p of the warp: block p / 4, quarter p % 4
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (base * 4 + p < nblocks * 4) v = __ldg(w + base * 4 + p);
+      stage[warp][(p >> 2) * kStageStride + (p & 3)] = v;
+    }
+    __syncwarp();
+    uint32_t word[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = stage[warp][lane * kStageStride + j];
+      word[4 * j] = v.x;
+      word[4 * j + 1] = v.y;
+      word[4 * j + 2] = v.z;
+      word[4 * j + 3] = v.w;
+    }
+    __syncwarp();
+    const int64_t blk = base + lane;
+    const bool valid = blk < nblocks;
+    const uint32_t sgn = (RHT && valid) ? __ldg(signs + col) : 0u;
+
+    double y[32];
+    uint32_t negbits = 0, nonfinite = 0;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      uint32_t b = (word[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
+      nonfinite |= ((b & 0x7F80u) == 0x7F80u) ? 1u : 0u;
+      if (RHT) {
+        b ^= ((sgn >> t) & 1u) << 15;
+      } else {
+        negbits |= (b >> 15) << t;
+      }
+      y[t] = bf16_to_f64(b);
+    }
+    if (RHT) {
+      // in-place fast Walsh-Hadamard transform, natural (Sylvester) order
+#pragma unroll
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if ((i & h) == 0) {
+            const double a = y[i], c = y[i + h];
+            y[i] = a + c;
+            y[i + h] = a - c;
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 32; ++t) negbits |= (y[t] < 0.0 ? 1u : 0u) << t;
+    }
+
+    // block maximum of |y| through the high words (magnitude order), then
+    // the significand test of the stochastic-rounding scale rule
+    uint32_t amax_hi = 0;
+#pragma unroll
+    for (int t = 0; t < 32; ++t)
+      amax_hi = max(amax_hi, static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu);
+    int sb = 0;
+    if (amax_hi != 0) {
+      sb = static_cast<int>(amax_hi >> 20) - 1023 + 125;
+      if (SR) {
+        const uint32_t frac_hi = amax_hi & 0xFFFFFu;
+        bool above = frac_hi > 0x80000u;
+        if (frac_hi == 0x80000u) {  // significand 1.5 in the high word: the low words decide
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            above |= (static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu) == amax_hi &&
+                     __double2loint(y[t]) != 0;
+        }
+        sb += above ? 1 : 0;
+      }
+      sb = min(max(sb, 0), 254);
+    }
+    const double inv_scale = __hiloint2double((127 - sb + 1023) << 20, 0);  // 2^(127 - sb)
+
+    uint32_t out[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint4 rnd = make_uint4(0u, 0u, 0u, 0u);
+      if (SR) {
+        const uint64_t ctr = static_cast<uint64_t>(blk) * 4 + g;  // (32 blk + 8 g) / 8
+        rnd = philox4x32_10(make_uint4(static_cast<uint32_t>(ctr), static_cast<uint32_t>(ctr >> 32),
+                                       0u, 0u),
+                            key0, key1);
+      }
+      const uint32_t rw[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+      uint32_t o = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int t = 8 * g + e;
+        const uint32_t u = (rw[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+        uint32_t c = e2m1_code<SR>(fabs(y[t]) * inv_scale, u);
+        c |= ((negbits >> t) & 1u) << 3;
+        o |= c << (4 * e);
+      }
+      out[g] = o;
+    }
+    if (valid) {
+      q[blk] = make_uint4(out[0], out[1], out[2], out[3]);
+      s[blk] = static_cast<uint8_t>(sb);
+      if (nonfinite) record_status(status, MOE_ERR_NONFINITE);
+    }
+    col += stride_mod;
+    if (col >= nbk) col -= nbk;
+  }
+}
+
+using KernelFn = void (*)(const uint4*, int64_t, int64_t, int64_t, const uint32_t*, uint32_t,
+                          uint32_t, uint4*, uint8_t*, int32_t*);
+
+KernelFn pick(uint32_t flags) {
+  switch (flags) {
+    case MOE_QUANT_RHT: return quantize_sr_rht_kernel<true, false>;
+    case MOE_QUANT_SR: return quantize_sr_rht_kernel<false, true>;
+    default: return quantize_sr_rht_kernel<true, true>;
+  }
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status mxfp4_quantize_sr_rht(const uint16_t* w_bf16, int64_t rows, int64_t K,
+                                            uint32_t flags, const uint32_t* rht_signs,
+                                            uint64_t seed, uint8_t* q_packed, uint8_t* scales,
+                                            int32_t* d_status, moe_stream stream) {
+  using namespace moe;
+  if (flags & ~static_cast<uint32_t>(MOE_QUANT_RHT | MOE_QUANT_SR)) return MOE_ERR_INVALID_ARG;
+  // no flag: the deterministic quantiser's bytes, from its own kernel
+  if (flags == 0) return mxfp4_quantize(w_bf16, rows, K, q_packed, scales, d_status, stream);
+  if (rows < 0 || K < 32 || (K % 32) != 0) return MOE_ERR_SHAPE;
+  if (rows > 0 && K > (int64_t(1) << 40) / rows) return MOE_ERR_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!w_bf16 || !q_packed || !scales) return MOE_ERR_INVALID_ARG;
+  if ((flags & MOE_QUANT_RHT) && !rht_signs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_bf16) || !aligned16(q_packed) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
+  if (rht_signs && (reinterpret_cast<uintptr_t>(rht_signs) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_device();
+  if (st != MOE_OK) return st;
+  const int64_t nblocks = rows * (K / 32);
+  const int64_t nbk = K / 32;
+  const int64_t want = (nblocks + kThreads - 1) / kThreads;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  const int64_t stride_mod = (static_cast<int64_t>(grid) * kThreads) % nbk;
+  pick(flags)<<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint4*>(w_bf16), nblocks, nbk, stride_mod, rht_signs,
+      static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
+      reinterpret_cast<uint4*>(q_packed), scales, d_status);
+  return launch_status();
+}

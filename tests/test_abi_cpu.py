@@ -23,7 +23,8 @@ def declared_functions():
 
 def test_header_declares_the_six_calls_and_helpers():
     names = declared_functions()
-    for n in ["mxfp4_quantize", "moe_route", "moe_permute", "moe_expert_mlp", "moe_combine",
+    for n in ["mxfp4_quantize", "mxfp4_quantize_sr_rht", "moe_route", "moe_permute",
+              "moe_expert_mlp", "moe_combine",
               "moe_layer_forward", "moe_workspace_size", "moe_status_string"]:
         assert n in names
 
@@ -116,3 +117,18 @@ def test_router_arguments_rejected_before_the_device():
     assert L.moe_router_topk(None, 16, 4, 128, 8, 4, None, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_router_topk(16, 24, 4, 128, 8, 4, None, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_router_topk(16, 16, 4, 128, 8, 4, 40, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_sr_rht_quantiser_arguments_rejected_before_the_device():
+    L = moe.lib
+    RHT, SR = moe.MOE_QUANT_RHT, moe.MOE_QUANT_SR
+    # (w, rows, K, flags, signs, seed, q, s, d_status, stream)
+    assert L.mxfp4_quantize_sr_rht(16, 4, 64, 4, 16, 0, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.mxfp4_quantize_sr_rht(16, 4, 48, SR, None, 0, 16, 16, None, None) == moe.MOE_ERR_SHAPE
+    assert L.mxfp4_quantize_sr_rht(16, -1, 64, SR, None, 0, 16, 16, None, None) == moe.MOE_ERR_SHAPE
+    assert L.mxfp4_quantize_sr_rht(16, 4, 64, RHT, None, 0, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.mxfp4_quantize_sr_rht(16, 4, 64, RHT, 18, 0, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.mxfp4_quantize_sr_rht(24, 4, 64, SR, None, 0, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.mxfp4_quantize_sr_rht(16, 4, 64, SR, None, 0, 16, 16, 18, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.mxfp4_quantize_sr_rht(None, 4, 64, 0, None, 0, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.mxfp4_quantize_sr_rht(16, 0, 64, RHT | SR, 16, 7, 16, 16, None, None) == moe.MOE_OK
