@@ -238,7 +238,10 @@ MOE_API moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x,
  *                arrays wgu_q and wdn_q 32-byte aligned
  *   h       out  [S][F] bf16 (caller-owned intermediate)
  *   y_perm  out  [S][D] bf16
- *   ws      in   device workspace of moe_workspace_size(shape, 1) bytes
+ *   ws      in   device workspace of moe_workspace_size(shape, 1) bytes,
+ *                16-byte aligned; its first 4 bytes are the device status
+ *                word, cleared by the call and set to MOE_ERR_TIMEOUT if a
+ *                bounded wait gave up (read it after the stream syncs)
  * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_WORKSPACE,
  * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA; device status MOE_ERR_TIMEOUT.      */
 MOE_API moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets,

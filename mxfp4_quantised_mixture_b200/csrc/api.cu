@@ -100,6 +100,9 @@ int sm_count() {
   return g_dev_sms[dev] > 0 ? g_dev_sms[dev] : 148;
 }
 
+// status head of the standalone expert-MLP workspace
+constexpr size_t kMlpStatusBytes = 256;
+
 bool shape_ok(const moe_shape& s) {
   if (s.T < 0 || s.T > (1 << 20)) return false;
   if (s.E < 1 || s.E > 256) return false;
@@ -121,7 +124,7 @@ size_t moe_workspace_size(moe_shape shape, int which) {
     case 0:
       return 0;
     case 1:
-      return expert_mlp_workspace(shape);
+      return kMlpStatusBytes + expert_mlp_workspace(shape);
     case 2:
       return layer_ws(shape).total;
     default:
@@ -162,12 +165,19 @@ moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, moe_sh
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (!aligned32(wgu_q) || !aligned32(wdn_q)) return MOE_ERR_INVALID_ARG;
-  const size_t need = expert_mlp_workspace(shape);
-  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return MOE_ERR_WORKSPACE;
+  // the first kMlpStatusBytes of ws hold the device status word, the rest
+  // is the GEMMs' workspace (same alignment class as ws itself)
+  const size_t need = kMlpStatusBytes + expert_mlp_workspace(shape);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   moe_status st = check_device();
   if (st != MOE_OK) return st;
-  return expert_mlp_launch(x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm, ws,
-                           nullptr, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return expert_mlp_launch(x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm,
+                           static_cast<char*>(ws) + kMlpStatusBytes, static_cast<int32_t*>(ws), s);
 }
 
 moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape shape,

@@ -28,7 +28,7 @@
 // Layout: one thread per 32-element block.  A warp loads 32 consecutive blocks
 // (2 KB) with coalesced 16-byte loads into a padded shared-memory stage (a
 // block's 64 bytes take 80, so the per-thread reads are free of bank
-// conflicts), decodes its own block into 32 doubles, transforms, encodes and
+// conflicts), widens its own block to 32 doubles, transforms, encodes and
 // writes its 16 code bytes (the warp's 512 are contiguous) and its scale byte.
 // The fp64 butterfly, Philox and the integer encoding make the kernel
 // instruction-bound rather than HBM-bound.
@@ -55,21 +55,6 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
     k1 += kPhiloxW1;
   }
   return c;
-}
-
-// exact fp64 value of a bf16 bit pattern (finite patterns; the exponent field
-// 0xFF gives some finite value, its block is reported as non-finite).  A zero
-// or subnormal m 2^-133 is (2^-81 + m 2^-133) - 2^-81, the first term built
-// from its bits, so no conversion instruction is needed.
-__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
-  const uint32_t e = (b >> 7) & 0xFFu, m = b & 0x7Fu;
-  double d;
-  if (e != 0)
-    d = __hiloint2double(static_cast<int>(((e + 896u) << 20) | (m << 13)), 0);
-  else
-    d = __hiloint2double(static_cast<int>(942u << 20), static_cast<int>(m)) - 0x1p-81;
-  return __hiloint2double(__double2hiint(d) | static_cast<int>((b & 0x8000u) << 16),
-                          __double2loint(d));
 }
 
 // E2M1 magnitude code of v = |y| / scale >= 0, from v's fp64 bit fields:
@@ -138,18 +123,16 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
     const bool valid = blk < nblocks;
     const uint32_t sgn = (RHT && valid) ? __ldg(signs + col) : 0u;
 
+    // bf16 -> fp32 bit pattern (a shift), the sign flip of the transform on
+    // its sign bit, then the exact widening to fp64 (subnormals included;
+    // Inf and NaN stay non-finite and are caught through the block maximum)
     double y[32];
-    uint32_t negbits = 0, nonfinite = 0;
 #pragma unroll
     for (int t = 0; t < 32; ++t) {
-      uint32_t b = (word[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
-      nonfinite |= ((b & 0x7F80u) == 0x7F80u) ? 1u : 0u;
-      if (RHT) {
-        b ^= ((sgn >> t) & 1u) << 15;
-      } else {
-        negbits |= (b >> 15) << t;
-      }
-      y[t] = bf16_to_f64(b);
+      const uint32_t wd = word[t >> 1];
+      uint32_t f = (t & 1) ? (wd & 0xFFFF0000u) : (wd << 16);
+      if (RHT) f ^= (sgn << (31 - t)) & 0x80000000u;
+      y[t] = static_cast<double>(__uint_as_float(f));
     }
     if (RHT) {
       // in-place fast Walsh-Hadamard transform, natural (Sylvester) order
@@ -164,8 +147,6 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
           }
         }
       }
-#pragma unroll
-      for (int t = 0; t < 32; ++t) negbits |= (y[t] < 0.0 ? 1u : 0u) << t;
     }
 
     // block maximum of |y| through the high words (magnitude order), then
@@ -174,6 +155,7 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
 #pragma unroll
     for (int t = 0; t < 32; ++t)
       amax_hi = max(amax_hi, static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu);
+    const bool nonfinite = amax_hi >= 0x7FF00000u;  // an Inf or NaN reached y
     int sb = 0;
     if (amax_hi != 0) {
       sb = static_cast<int>(amax_hi >> 20) - 1023 + 125;
@@ -209,7 +191,10 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
         const int t = 8 * g + e;
         const uint32_t u = (rw[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
         uint32_t c = e2m1_code<SR>(fabs(y[t]) * inv_scale, u);
-        c |= ((negbits >> t) & 1u) << 3;
+        // sign bit: that of x without the transform (-0 included); with it,
+        // y < 0 only (a high word above 0x80000000 is a negative nonzero)
+        const uint32_t hy = static_cast<uint32_t>(__double2hiint(y[t]));
+        c |= (RHT ? (hy > 0x80000000u ? 1u : 0u) : (hy >> 31)) << 3;
         o |= c << (4 * e);
       }
       out[g] = o;

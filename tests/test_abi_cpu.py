@@ -60,6 +60,8 @@ def test_workspace_size_is_host_only_and_monotone():
     # the layer workspace holds at least x_perm, h and y_perm (bf16)
     assert b >= S * 2880 * 2 * 3
     assert moe.moe_workspace_size(small, 9) == 0
+    # the standalone expert MLP's workspace starts with a 256-byte status head
+    assert moe.moe_workspace_size(small, moe.WS_EXPERT_MLP) >= 256
     assert moe.moe_workspace_size(moe.make_shape(64, 300, 4, 2880, 2880), moe.WS_LAYER) == 0
 
 

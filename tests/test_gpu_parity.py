@@ -188,9 +188,11 @@ def test_expert_mlp_and_combine_tiny(dev):
     h = torch.empty((S, wl.d_ff), dtype=torch.bfloat16, device=dev)
     y = torch.empty((S, wl.d_model), dtype=torch.bfloat16, device=dev)
     ws = moe.alloc_workspace(L.shape, moe.WS_EXPERT_MLP, dev)
+    ws[:4].fill_(0xFF)  # the call clears its status word
     moe.moe_expert_mlp(to_dev_u16(xp, dev), torch.from_numpy(offsets).to(dev), L.shape, L.wgu_q,
                        L.wgu_s, L.wdn_q, L.wdn_s, h, y, ws)
     torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == moe.MOE_OK
     assert_layer_close(bf16_np(h), oh, "h")
     # y mixes bf16 h values: a flip of one h moves y by far less than an ulp
     assert_layer_close(bf16_np(y), oy, "y")
