@@ -134,3 +134,29 @@ def test_sr_rht_quantiser_arguments_rejected_before_the_device():
     assert L.mxfp4_quantize_sr_rht(16, 4, 64, SR, None, 0, 16, 16, 18, None) == moe.MOE_ERR_INVALID_ARG
     assert L.mxfp4_quantize_sr_rht(None, 4, 64, 0, None, 0, 16, 16, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.mxfp4_quantize_sr_rht(16, 0, 64, RHT | SR, 16, 7, 16, 16, None, None) == moe.MOE_OK
+
+
+def _no_gpu_here() -> bool:
+    import torch
+
+    return not torch.cuda.is_available() and not os.path.exists("/dev/nvidiactl")
+
+
+@pytest.mark.skipif(not _no_gpu_here(), reason="its placeholder pointers must never reach a device")
+def test_well_formed_calls_fail_cleanly_without_a_device():
+    # host-side failure injection: every argument passes validation, the
+    # device probe finds no usable GPU, and the call returns a status with
+    # nothing launched (no crash, no fallback)
+    L = moe.lib
+    sh = moe.make_shape(64, 32, 4, 2880, 2880)
+    need = moe.moe_workspace_size(sh, moe.WS_LAYER)
+    mlp = moe.moe_workspace_size(sh, moe.WS_EXPERT_MLP)
+    no_device = (moe.MOE_ERR_CUDA, moe.MOE_ERR_UNSUPPORTED)
+    assert L.mxfp4_quantize(16, 4, 64, 16, 16, None, None) in no_device
+    assert L.mxfp4_quantize_sr_rht(16, 4, 64, moe.MOE_QUANT_SR, None, 1, 16, 16, None, None) in no_device
+    assert L.moe_route(16, 4, 32, 4, 16, 16, None) in no_device
+    assert L.moe_router_topk(16, 16, 4, 128, 8, 4, None, 16, 16, None, None) in no_device
+    assert L.moe_permute(16, 16, sh, 16, 16, 16, 16, 16, None, 0, None) in no_device
+    assert L.moe_expert_mlp(16, 16, sh, 32, 16, 32, 16, 16, 16, 256, mlp, None) in no_device
+    assert L.moe_combine(16, 16, 16, sh, 16, None) in no_device
+    assert L.moe_layer_forward(16, 16, sh, 32, 16, 32, 16, 16, 256, need, None) in no_device
