@@ -82,10 +82,17 @@ lib = _load()
 
 
 def _p(t) -> int | None:
+    """Device pointer of a tensor argument (None and raw integer addresses
+    pass through).  The C ABI reads dense row-major device arrays, so a
+    strided view or a host tensor is refused here rather than misread."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous (dense row-major)")
     return t.data_ptr()
 
 

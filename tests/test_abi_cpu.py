@@ -160,3 +160,18 @@ def test_well_formed_calls_fail_cleanly_without_a_device():
     assert L.moe_expert_mlp(16, 16, sh, 32, 16, 32, 16, 16, 16, 256, mlp, None) in no_device
     assert L.moe_combine(16, 16, 16, sh, 16, None) in no_device
     assert L.moe_layer_forward(16, 16, sh, 32, 16, 32, 16, 16, 256, need, None) in no_device
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    import torch
+
+    sh = moe.make_shape(4, 8, 4, 128, 128)
+    host = torch.zeros((4, 8), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        moe.moe_route(host, 4, host, host)
+    with pytest.raises(ValueError):
+        moe.moe_combine(host, host, host, sh, host)
+    if torch.cuda.is_available():  # a strided device view is refused as well
+        dev = torch.zeros((8, 4), dtype=torch.float32, device="cuda").t()
+        with pytest.raises(ValueError):
+            moe.moe_route(dev, 4, dev, dev)
