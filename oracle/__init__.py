@@ -72,6 +72,8 @@ def _L():
         lib.oracle_gather.argtypes = [vp, vp, i64, i32, i32, vp]
         lib.oracle_expert_mlp.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32]
         lib.oracle_expert_mlp.restype = i32
+        lib.oracle_expert_mlp_bf16.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, i32]
+        lib.oracle_expert_mlp_bf16.restype = i32
         lib.oracle_combine.argtypes = [vp, vp, vp, i64, i32, i32, vp]
         lib.oracle_layer_forward.argtypes = [vp, vp, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32]
         lib.oracle_layer_forward.restype = i32
@@ -245,6 +247,26 @@ def expert_mlp(x_perm, offsets, wgu_q, wgu_s, wdn_q, wdn_s, want_h: bool = True)
                                 _p(h) if want_h else None, _p(y), _threads())
     if rc != 0:
         raise MemoryError("oracle_expert_mlp: allocation failed")
+    return h, y
+
+
+def expert_mlp_bf16(x_perm, offsets, wgu_bf16, wdn_bf16, want_h: bool = True):
+    """The grouped expert MLP with unquantised bf16 weights (bit patterns):
+    wgu [E][2F][D], wdn [E][D][F] -> (h [S][F] or None, y [S][D])."""
+    xp = _c(x_perm, np.uint16)
+    off = _c(offsets, np.int32)
+    E = off.size - 1
+    S, D = xp.shape
+    F = wdn_bf16.shape[-1]
+    gu = _c(wgu_bf16, np.uint16)
+    dn = _c(wdn_bf16, np.uint16)
+    assert gu.shape == (E, 2 * F, D) and dn.shape == (E, D, F)
+    h = np.empty((S, F), dtype=np.uint16) if want_h else None
+    y = np.empty((S, D), dtype=np.uint16)
+    rc = _L().oracle_expert_mlp_bf16(_p(xp), _p(off), E, D, F, _p(gu), _p(dn),
+                                     _p(h) if want_h else None, _p(y), _threads())
+    if rc != 0:
+        raise MemoryError("oracle_expert_mlp_bf16: allocation failed")
     return h, y
 
 

@@ -583,6 +583,37 @@ int oracle_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, int E, int
   return 0;
 }
 
+/* The same grouped expert MLP with unquantised bf16 weights, the comparison
+ * point the pages set against MXFP4 (the bf16 path takes about 4x the
+ * memory: "Tricks from OpenAI gpt-oss ...", section 7; agentlenshq (ja),
+ * "What is MXFP4").  Weights: wgu [E][2F][D], wdn [E][D][F] as bf16 bit
+ * patterns; every step as in oracle_expert_mlp, the weights taken at their
+ * exact bf16 values instead of decoded codes. */
+int oracle_expert_mlp_bf16(const uint16_t* x_perm, const int32_t* offsets, int E, int D, int F,
+                           const uint16_t* wgu_bf16, const uint16_t* wdn_bf16, uint16_t* h,
+                           uint16_t* y, int nthreads) {
+  double* wgu = (double*)malloc(sizeof(double) * 2 * (size_t)F * D);
+  double* wdn = (double*)malloc(sizeof(double) * (size_t)D * F);
+  if (!wgu || !wdn) {
+    free(wgu);
+    free(wdn);
+    return -1;
+  }
+  for (int e = 0; e < E; ++e) {
+    int64_t r0 = offsets[e], r1 = offsets[e + 1];
+    if (r1 <= r0) continue;
+    const uint16_t* gsrc = wgu_bf16 + (int64_t)e * 2 * F * D;
+    const uint16_t* dsrc = wdn_bf16 + (int64_t)e * D * F;
+    for (int64_t i = 0; i < 2 * (int64_t)F * D; ++i) wgu[i] = oracle_bf16_value(gsrc[i]);
+    for (int64_t i = 0; i < (int64_t)D * F; ++i) wdn[i] = oracle_bf16_value(dsrc[i]);
+    expert_rows_parallel(x_perm + r0 * D, r1 - r0, D, F, wgu, wdn, h ? h + r0 * F : NULL,
+                         y + r0 * D, nthreads);
+  }
+  free(wgu);
+  free(wdn);
+  return 0;
+}
+
 /* out[t][d] = bf16( sum_j w[t][j] * y_perm[slot_pos[t*k+j]][d] ), j ascending */
 void oracle_combine(const uint16_t* y_perm, const int32_t* slot_pos, const double* w, int64_t T,
                     int k, int D, uint16_t* out) {

@@ -515,3 +515,57 @@ def test_router_row_permutation_permutes_columns():
     w = syn.normal_bf16(23, 904, (E, D), sigma=0.05)
     perm = np.array([4, 8, 0, 3, 1, 7, 2, 6, 5])
     assert np.array_equal(oracle.router_logits(x, w[perm]), oracle.router_logits(x, w)[:, perm])
+
+
+# ------------------------------------------------ bf16 expert path (comparison)
+
+
+def _bf16_bits_exact(v: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of values known to be bf16-representable."""
+    f32 = v.astype(np.float32)
+    assert np.array_equal(f32.astype(np.float64), v)
+    bits = (f32.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(bits_to_f64(bits), v)  # nothing below bf16 precision was dropped
+    return bits
+
+
+def test_bf16_expert_mlp_equals_mxfp4_on_decoded_weights():
+    # every MXFP4 value at these scales is a bf16 value, so the bf16 path fed
+    # the decoded weights must give the MXFP4 path's h and y bit for bit
+    wl = syn.Workload("cmp", T=21, d_model=128, d_ff=192, E=4, k=2, seed=12)
+    x = syn.activations(wl)
+    lg = syn.logits(wl)
+    gq, gs, dq, ds = _tiny_quantised(wl)
+    idx, _ = oracle.route(lg, wl.k)
+    _, offsets, sorted_slot, _ = oracle.permute(idx, wl.E)
+    xp = oracle.gather(x, sorted_slot, wl.k)
+    h1, y1 = oracle.expert_mlp(xp, offsets, gq, gs, dq, ds)
+    gu16 = _bf16_bits_exact(oracle.mxfp4_decode(gq, gs))
+    dn16 = _bf16_bits_exact(oracle.mxfp4_decode(dq, ds))
+    h2, y2 = oracle.expert_mlp_bf16(xp, offsets, gu16, dn16)
+    assert np.array_equal(h1, h2) and np.array_equal(y1, y2)
+
+
+def test_bf16_single_expert_is_dense_mlp():
+    # unquantised bf16 weights (not MXFP4 values): one expert against a dense
+    # fp64 torch restatement, up to ties of the bf16 roundings
+    T, D, F = 11, 128, 64
+    x = syn.normal_bf16(31, 1, (T, D), sigma=1.0)
+    gu = syn.normal_bf16(31, 3, (1, 2 * F, D), sigma=0.05)
+    dn = syn.normal_bf16(31, 4, (1, D, F), sigma=0.05)
+    offsets = np.array([0, T], dtype=np.int32)
+    h, y = oracle.expert_mlp_bf16(x, offsets, gu, dn)
+    X = torch.from_numpy(bits_to_f64(x))
+    Wg = torch.from_numpy(bits_to_f64(gu[0]))
+    Wd = torch.from_numpy(bits_to_f64(dn[0]))
+    G = X @ Wg[:F].T
+    U = X @ Wg[F:].T
+    H = np_round_bf16((torch.nn.functional.silu(G) * U).numpy())
+    Y = np_round_bf16((torch.from_numpy(H) @ Wd.T).numpy())
+    assert np.array_equal(bits_to_f64(h), H)
+    assert np.array_equal(bits_to_f64(y), Y)
+    # a planted sign error in one weight changes the output
+    gu2 = gu.copy()
+    gu2[0, 0, 0] ^= 0x8000
+    _, y_bad = oracle.expert_mlp_bf16(x, offsets, gu2, dn)
+    assert not np.array_equal(y_bad, y)
