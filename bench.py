@@ -19,6 +19,12 @@ once, before timing, by the library's mxfp4_quantize.  L2 is flushed (a
   whichever roofline term of the call is larger.
 * cpu_baseline: the fp64 CPU oracle, as it stands, on the host cores, over a
   bounded sample of the same workload (rank 0, one GPU only).
+* router: moe_router_topk (router scores fused with the top-k) on the same
+  tokens against a seeded router matrix.
+* quantize: the quantisers timed on their own (mxfp4_quantize, and
+  mxfp4_quantize_sr_rht with the random-sign Hadamard transform and
+  stochastic rounding) over the first chunk of the workload's bf16 gate/up
+  weights, GB/s of algorithmic bytes against the HBM copy peak.
 Under torchrun each rank runs its own replica of the workload on its own GPU
 (independent token batches, no collective on the data path): weak scaling.
 """
