@@ -12,7 +12,7 @@ import torch
 import mxfp4_quantised_mixture_b200 as moe
 import oracle
 import synthetic as syn
-from layer_cases import (ROUTE_W_ATOL, assert_layer_close, bf16_np, bf16_ulp, device_layer,
+from layer_cases import (ROUTE_W_ATOL, assert_layer_close, bf16_np, device_layer,
                          oracle_layer_with_y, oracle_tokens_with_y, oracle_weights_for, run_layer,
                          to_dev_u16)
 
