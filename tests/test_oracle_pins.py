@@ -569,3 +569,21 @@ def test_bf16_single_expert_is_dense_mlp():
     gu2[0, 0, 0] ^= 0x8000
     _, y_bad = oracle.expert_mlp_bf16(x, offsets, gu2, dn)
     assert not np.array_equal(y_bad, y)
+
+
+@pytest.mark.parametrize("T,E,k", [(64, 32, 4), (128, 128, 4), (50, 8, 8), (20, 3, 1)])
+def test_route_invariants(T, E, k):
+    # token-choice top-k with the softmax over the chosen k ("Welcome GPT OSS
+    # ...", section 4): k distinct experts per token, weights in (0, 1]
+    # summing to 1 and ordered like their logits
+    lg = np.random.default_rng(T * E + k).standard_normal((T, E)).astype(np.float32)
+    idx, w = oracle.route(lg, k)
+    for t in range(T):
+        assert len(set(idx[t].tolist())) == k
+        assert abs(w[t].sum() - 1.0) <= 1e-15
+        assert (w[t] > 0).all() and (np.diff(w[t]) <= 0).all()
+        assert (np.diff(lg[t, idx[t]].astype(np.float64)) <= 0).all()
+        # every unchosen logit is at most the smallest chosen one
+        rest = np.setdiff1d(np.arange(E), idx[t])
+        if rest.size:
+            assert lg[t, rest].max() <= lg[t, idx[t]].min()
