@@ -8,25 +8,37 @@ synthetic tokens with the workload's shapes; the MXFP4 weights are quantised
 once, before timing, by the library's mxfp4_quantize.  L2 is flushed (a
 256 MiB device write) before every timed step, outside the timed events.
 
+The line's own fields are the largest single-GPU workload, the skewed
+120B-shaped prefill batch (T 16384, E 128); ``per_workload`` carries the same
+fields for the other four workloads (tiny, 20B decode, 20B prefill, 120B
+decode), timed in the same run.  ``--workload NAME`` times that one alone.
+
 * value: tokens/s of the whole job (all ranks), inputs resident in HBM, from
   CUDA events around each step on the launching stream, max over ranks.
 * e2e: the same metric through the same C-ABI call with host buffers: the
   step's x and logits are copied from pinned host memory and the output is
   copied back inside the timed region.
 * roofline: the grouped expert MLP (moe_expert_mlp: the GEMM launches that
-  dominate the step), algorithmic bytes (or FLOPs) per call / its event time,
-  against the measured HBM copy bandwidth (or the measured bf16 tensor rate),
-  whichever roofline term of the call is larger.
-* cpu_baseline: the fp64 CPU oracle, as it stands, on the host cores, over a
-  bounded sample of the same workload (rank 0, one GPU only).
-* router: moe_router_topk (router scores fused with the top-k) on the same
-  tokens against a seeded router matrix.
+  dominate the step, with the tile plan and, on the block-scaled path, the
+  split of the input rows), algorithmic bytes (or FLOPs) per call / its event
+  time, against the measured HBM copy bandwidth (or the measured bf16 tensor
+  rate), whichever roofline term of the call is larger.
+* cpu_baseline: the fp64 CPU oracle, as it stands, on the host cores, over
+  the first 64 tokens of the batch (all of them when it has fewer), with the
+  weights of the experts they route to quantised beforehand (rank 0, one GPU
+  only).  The reference arm times the same sample per step.
+* router: moe_router_topk (router scores fused with the top-k) on the
+  headline workload's tokens against a seeded router matrix.
+* unquantised: at the 20B decode batch, the grouped expert MLP on the
+  unquantised bf16 weights (moe_expert_mlp_unquantised) beside the MXFP4 one,
+  weight bytes streamed and time of each.
 * quantize: the quantisers timed on their own (mxfp4_quantize, and
   mxfp4_quantize_sr_rht with the random-sign Hadamard transform and
-  stochastic rounding) over the first chunk of the workload's bf16 gate/up
-  weights, GB/s of algorithmic bytes against the HBM copy peak.
-Under torchrun each rank runs its own replica of the workload on its own GPU
-(independent token batches, no collective on the data path): weak scaling.
+  stochastic rounding) over the first chunk of the headline workload's bf16
+  gate/up weights, GB/s of algorithmic bytes against the HBM copy peak.
+Under torchrun each rank runs its own replica of every workload on its own
+GPU (independent token batches, no collective on the data path): weak
+scaling.
 """
 from __future__ import annotations
 
@@ -49,26 +61,22 @@ import synthetic as syn  # noqa: E402
 
 METRIC = "MoE-layer tokens/s on 1 B200; % of roofline (HBM GB/s decode, TC TFLOP/s prefill)"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "20b_decode"
+HEADLINE = "120b_skewed_prefill"
+OTHERS = ["120b_decode", "20b_decode", "20b_prefill", "tiny"]
 FLUSH_BYTES = 256 << 20
-# kernel launches of one moe_layer_forward call: route, permute (bookkeeping +
-# row gather), expert MLP, combine.  The expert MLP is a tile plan and two
-# GEMMs, plus the activation and intermediate splits on the block-scaled path
-# that the library takes when twice the mean routed rows per expert is <= 64.
+CPU_SAMPLE_TOKENS = 64
+# the unquantised (bf16 weight) expert MLP is timed beside the MXFP4 one here
+UNQUANTISED_AT = "20b_decode"
+# kernel launches of one moe_layer_forward call: route, permute (with the
+# GEMMs' tile list), the row gather (or, on the block-scaled path, the split
+# of the rows straight from x), the gate/up GEMM, the down GEMM, combine
+LAUNCHES_PER_LAYER = 6
 
-
-def launches_per_layer(T: int, E: int, k: int) -> int:
-    S = T * k
-    block_scaled = 2 * ((S + E - 1) // E) <= 64
-    return 9 if block_scaled else 7
-
-
-# dram bytes (read + write) of one moe_expert_mlp call on the default workload,
-# from an ncu capture of the kernels whose code (comments and whitespace aside)
-# hashes to TRAFFIC_SRC_SHA; reported only while that code is unchanged
-TRAFFIC_BYTES = 438201856  # gate/up 285.19 + 4.95 MB, down 144.21 + 3.86 MB (read + write)
-TRAFFIC_SRC_SHA = "dfc92b05a77c321f"
-TRAFFIC_WORKLOAD = DEFAULT_WORKLOAD
+# dram bytes (read + write) of one moe_expert_mlp call per workload, from ncu
+# captures of the kernels whose code (comments and whitespace aside) hashes
+# to TRAFFIC_SRC_SHA; reported only while that code is unchanged
+TRAFFIC_BYTES: dict[str, int] = {}
+TRAFFIC_SRC_SHA = ""
 
 
 def parse():
@@ -76,7 +84,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(syn.WORKLOADS),
+                    help="time this workload alone (default: the headline and all others)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -106,8 +115,11 @@ def code_tokens(src: str) -> str:
 
 
 def kernel_src_sha() -> str:
-    with open(os.path.join(ROOT, "mxfp4_quantised_mixture_b200", "csrc", "expert_mlp.cu")) as f:
-        return hashlib.sha256(code_tokens(f.read()).encode()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for name in ("expert_mlp.cu", "expert_mlp_bf16.cu"):
+        with open(os.path.join(ROOT, "mxfp4_quantised_mixture_b200", "csrc", name)) as f:
+            h.update(code_tokens(f.read()).encode())
+    return h.hexdigest()[:16]
 
 
 # ------------------------------------------------------------------ clocks
@@ -177,57 +189,80 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(mhz)}
 
 
-# ------------------------------------------------------------- reference arm
+# --------------------------------------------------- oracle (CPU baseline)
 
 
-def cpu_oracle_sample(wl, n_tokens: int, weights=None):
-    """Time the fp64 oracle over the first n_tokens of the workload.
-    Returns (seconds, tokens, threads, weights)."""
+def oracle_weights(wl, tokens):
+    """Oracle-quantised weights [E][...] of the experts the tokens route to
+    (the others zero), made before any timing."""
     import oracle
 
-    x = syn.activations(wl)
     lg = syn.logits(wl)
+    idx, _ = oracle.route(lg[tokens], wl.k)
+    need = sorted(set(int(v) for v in idx.ravel()))
+    D, F, E = wl.d_model, wl.d_ff, wl.E
+    gq = np.zeros((E, 2 * F, D // 2), np.uint8)
+    gs = np.zeros((E, 2 * F, D // 32), np.uint8)
+    dq = np.zeros((E, D, F // 2), np.uint8)
+    ds = np.zeros((E, D, F // 32), np.uint8)
+    for e in need:
+        q, s = oracle.quantize_experts(syn.w_gate_up(wl, [e]))
+        gq[e], gs[e] = q[0], s[0]
+        q, s = oracle.quantize_experts(syn.w_down(wl, [e]))
+        dq[e], ds[e] = q[0], s[0]
+    return gq, gs, dq, ds
+
+
+def cpu_oracle_sample(wl, n_tokens: int, weights=None, inputs=None):
+    """Time the fp64 oracle over the first n_tokens of the workload (the
+    whole layer when that is all of them).  Returns (seconds, tokens,
+    threads, weights, inputs)."""
+    import oracle
+
+    if inputs is None:
+        inputs = (syn.activations(wl), syn.logits(wl))
+    x, lg = inputs
     tokens = list(range(min(n_tokens, wl.T)))
     if weights is None:
-        idx, _ = oracle.route(lg[tokens], wl.k)
-        need = sorted(set(int(v) for v in idx.ravel()))
-        D, F, E = wl.d_model, wl.d_ff, wl.E
-        gq = np.zeros((E, 2 * F, D // 2), np.uint8)
-        gs = np.zeros((E, 2 * F, D // 32), np.uint8)
-        dq = np.zeros((E, D, F // 2), np.uint8)
-        ds = np.zeros((E, D, F // 32), np.uint8)
-        for e in need:
-            q, s = oracle.quantize_experts(syn.w_gate_up(wl, [e]))
-            gq[e], gs[e] = q[0], s[0]
-            q, s = oracle.quantize_experts(syn.w_down(wl, [e]))
-            dq[e], ds[e] = q[0], s[0]
-        weights = (gq, gs, dq, ds)
+        weights = oracle_weights(wl, tokens)
     t0 = time.perf_counter()
     if len(tokens) == wl.T:
         oracle.layer_forward(x, lg, wl.k, *weights)
     else:
         oracle.layer_tokens(x, lg, wl.k, *weights, tokens)
     dt = time.perf_counter() - t0
-    return dt, len(tokens), max(1, min(64, os.cpu_count() or 1)), weights
+    return dt, len(tokens), max(1, min(64, os.cpu_count() or 1)), weights, inputs
 
 
-def reference_sample_tokens(wl) -> int:
-    return min(wl.T, 4)
+def sample_label(wl, n: int) -> str:
+    what = f"all {n} tokens of the batch" if n == wl.T else f"first {n} of {wl.T} tokens"
+    return (what + "; the oracle's weights of the experts they route to quantised before timing, "
+            "their decode to fp64 inside each timed call")
+
+
+def cpu_baseline(wl) -> dict:
+    n = min(wl.T, CPU_SAMPLE_TOKENS)
+    dt, tok, threads, weights, inputs = cpu_oracle_sample(wl, n)
+    times = [dt]
+    while sum(times) < 10.0 and len(times) < 5:  # about 10 s of CPU work
+        times.append(cpu_oracle_sample(wl, n, weights, inputs)[0])
+    return {"value": tok / statistics.mean(times), "unit": UNIT, "cores": threads,
+            "kind": "oracle", "sample": sample_label(wl, tok) + f"; mean of {len(times)} calls"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = syn.WORKLOADS[args.workload]
-    n = reference_sample_tokens(wl)
-    weights = None
+    wl = syn.WORKLOADS[args.workload or HEADLINE]
+    n = min(wl.T, CPU_SAMPLE_TOKENS)
+    weights = inputs = None
     for _ in range(args.warmup):
-        _, _, _, weights = cpu_oracle_sample(wl, n, weights)
+        _, _, _, weights, inputs = cpu_oracle_sample(wl, n, weights, inputs)
     total = 0.0
     threads = 1
     for _ in range(args.steps):
-        dt, tok, threads, weights = cpu_oracle_sample(wl, n, weights)
+        dt, tok, threads, weights, inputs = cpu_oracle_sample(wl, n, weights, inputs)
         total += dt
     value = args.steps * n / total
     line = {
@@ -237,8 +272,7 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(wl),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{n} of {wl.T} tokens per step, first tokens of the batch, "
-                                   "weights of the experts they route to quantised before timing"},
+                         "sample": sample_label(wl, n) + ", per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -317,63 +351,91 @@ def quantiser_timings(moe, w, flush, stream, steps, hbm):
     return out
 
 
-def run_ours(args):
+class Ctx:
+    """Device, stream, flush buffer and rank layout shared by the workloads."""
+
+    def __init__(self, args):
+        import torch
+        import torch.distributed as dist
+
+        self.args = args
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world > 1:
+            import datetime
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+        self.dev = torch.device("cuda", self.local)
+        torch.cuda.set_device(self.dev)
+        self.stream = torch.cuda.current_stream(self.dev)
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=self.dev)
+        self.peaks = peaks()
+
+    def barrier(self):
+        import torch.distributed as dist
+
+        if self.world > 1:
+            dist.barrier()
+
+
+def quantised_weights(moe, ctx, wl, keep_first_chunk=False, keep_bf16=False):
+    """The workload's MXFP4 weights on the device, quantised by the library
+    from the seeded bf16 weights (generated on the host a chunk of experts at
+    a time); with keep_bf16 also the bf16 weights themselves."""
     import torch
-    import torch.distributed as dist
 
-    import mxfp4_quantised_mixture_b200 as moe
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    wl = syn.WORKLOADS[args.workload]
-    D, F, E, T, k = wl.d_model, wl.d_ff, wl.E, wl.T, wl.k
-    S = T * k
-    shape = moe.make_shape(T, E, k, D, F)
-
-    # ---- inputs (seeded, synthetic) and weights quantised by the library
-    x_np = syn.activations(wl)
-    lg_np = syn.logits(wl)
-    x = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
-    logits = torch.from_numpy(lg_np).to(dev)
+    dev = ctx.dev
+    D, F, E = wl.d_model, wl.d_ff, wl.E
     wgu_q = torch.empty((E, 2 * F, D // 2), dtype=torch.uint8, device=dev)
     wgu_s = torch.empty((E, 2 * F, D // 32), dtype=torch.uint8, device=dev)
     wdn_q = torch.empty((E, D, F // 2), dtype=torch.uint8, device=dev)
     wdn_s = torch.empty((E, D, F // 32), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     chunk = max(1, min(E, (1 << 28) // (2 * F * D)))
+    first = None
+    if keep_bf16:
+        bf_gu = torch.empty((E, 2 * F, D), dtype=torch.bfloat16, device=dev)
+        bf_dn = torch.empty((E, D, F), dtype=torch.bfloat16, device=dev)
     for e0 in range(0, E, chunk):
         ex = list(range(e0, min(E, e0 + chunk)))
         gu = torch.from_numpy(syn.w_gate_up(wl, ex).view(np.int16)).to(dev).view(torch.bfloat16)
         dn = torch.from_numpy(syn.w_down(wl, ex).view(np.int16)).to(dev).view(torch.bfloat16)
         moe.mxfp4_quantize(gu, wgu_q[e0:e0 + len(ex)], wgu_s[e0:e0 + len(ex)], status)
         moe.mxfp4_quantize(dn, wdn_q[e0:e0 + len(ex)], wdn_s[e0:e0 + len(ex)], status)
-        if e0 == 0:
-            gu_first = gu  # kept for the quantiser timings below
+        if e0 == 0 and keep_first_chunk:
+            first = gu
+        if keep_bf16:
+            bf_gu[e0:e0 + len(ex)].copy_(gu)
+            bf_dn[e0:e0 + len(ex)].copy_(dn)
         del gu, dn
     torch.cuda.synchronize()
     if int(status.item()) != 0:
         raise RuntimeError("quantiser reported non-finite weights")
+    return (wgu_q, wgu_s, wdn_q, wdn_s), {"first": first,
+                                          "bf16": (bf_gu, bf_dn) if keep_bf16 else None}
 
+
+def measure_workload(moe, ctx, wl, weights) -> dict:
+    """Time one workload: the layer step, the expert MLP's roofline, e2e."""
+    import torch
+
+    args, dev, stream, flush = ctx.args, ctx.dev, ctx.stream, ctx.flush
+    D, F, E, T, k = wl.d_model, wl.d_ff, wl.E, wl.T, wl.k
+    S = T * k
+    shape = moe.make_shape(T, E, k, D, F)
+    wgu_q, wgu_s, wdn_q, wdn_s = weights
+    x_np = syn.activations(wl)
+    lg_np = syn.logits(wl)
+    x = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    logits = torch.from_numpy(lg_np).to(dev)
     out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
     ws = moe.alloc_workspace(shape, moe.WS_LAYER, dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def layer():
         moe.moe_layer_forward(x, logits, shape, wgu_q, wgu_s, wdn_q, wdn_s, out, ws, stream)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -385,10 +447,10 @@ def run_ours(args):
     # ---- timed region: K steps, events around each step, L2 flushed between
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(ctx.local)
     clocks.start()
     time.sleep(0.3)
-    barrier()
+    ctx.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for i in range(args.steps):
@@ -397,13 +459,15 @@ def run_ours(args):
         layer()
         ends[i].record(stream)
     torch.cuda.synchronize()
-    barrier()
+    ctx.barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
+    if int(ws[:4].view(torch.int32).item()) != 0:
+        raise RuntimeError("layer reported device status %d" % int(ws[:4].view(torch.int32).item()))
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = reduce_max(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
-    value = job_throughput(world, T, args.steps, total_ms)
+    value = job_throughput(ctx.world, T, args.steps, total_ms)
 
     # ---- roofline of the grouped expert MLP: the same step through the
     #      individual calls, with events around moe_expert_mlp
@@ -433,7 +497,7 @@ def run_ours(args):
     mlp_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(m_starts, m_ends))
     touched = int((counts > 0).sum().item())
     mlp_bytes = touched * expert_bytes(wl) + 2 * S * D * 2
-    hbm, tc_burst, tc_sust, peak_kind = peaks()
+    hbm, tc_burst, tc_sust, peak_kind = ctx.peaks
     mlp_flops = 6.0 * S * D * F
     # the bound is whichever roofline term is larger for this call: the bytes
     # at the measured copy bandwidth or the FLOPs at the measured bf16 rate
@@ -446,43 +510,14 @@ def run_ours(args):
         roof = {"bound": "hbm", "achieved": mlp_bytes / (mlp_ms / 1e3) / 1e9, "peak": hbm,
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    traffic = TRAFFIC_BYTES if (TRAFFIC_BYTES is not None and TRAFFIC_SRC_SHA == kernel_src_sha()
-                                and args.workload == TRAFFIC_WORKLOAD) else None
+    traffic = TRAFFIC_BYTES.get(wl.name) if TRAFFIC_SRC_SHA == kernel_src_sha() else None
+    roof.update(traffic=traffic, kernel="moe_expert_mlp (grouped gate/up+SwiGLU and down GEMMs)",
+                algorithmic_bytes=mlp_bytes, ms=mlp_ms, peak_source=peak_kind,
+                path="block-scaled" if 2 * -(-S // E) <= 64 else "bf16-decode")
     layer_bytes = touched * expert_bytes(wl) + T * D * 2 + T * E * 4 + T * D * 2
     layer_flops = 6.0 * S * D * F
     t_roof_meas = max(layer_bytes / (hbm * 1e9), layer_flops / (tc_sust * 1e12))
     t_roof_spec = max(layer_bytes / 8e12, layer_flops / 2.25e15)
-
-    # ---- router scores fused with the top-k (moe_router_topk) on the same
-    #      tokens, against a seeded bf16 router matrix [E][D]
-    router = None
-    if D % 64 == 0:
-        w_router = torch.from_numpy(syn.normal_bf16(wl.seed, 40, (E, D), sigma=1.0 / D ** 0.5)
-                                    .view(np.int16)).to(dev).view(torch.bfloat16)
-        r_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-        r_w = torch.empty((T, k), dtype=torch.float32, device=dev)
-        r_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        r_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        for i in range(args.steps + 2):
-            flush.fill_(i & 0xFF)
-            if i >= 2:
-                r_starts[i - 2].record(stream)
-            moe.moe_router_topk(x, w_router, k, r_idx, r_w, None, None, stream)
-            if i >= 2:
-                r_ends[i - 2].record(stream)
-        torch.cuda.synchronize()
-        r_ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in zip(r_starts, r_ends))
-        r_bytes = T * D * 2 + E * D * 2 + T * k * 8
-        router = {"call": "moe_router_topk", "ms": r_ms, "bytes": r_bytes,
-                  "GB/s": r_bytes / (r_ms / 1e3) / 1e9,
-                  "TFLOP/s": 2.0 * T * D * E / (r_ms / 1e3) / 1e12}
-
-    # ---- the quantisers, timed on their own over the first chunk of gate/up
-    #      weights (bf16 in, larger than L2): the deterministic one that
-    #      produced the layer's weights, and the training-style one with the
-    #      random-sign Hadamard transform and stochastic rounding
-    quant = quantiser_timings(moe, gu_first, flush, stream, args.steps, hbm)
-    del gu_first
 
     # ---- end to end through the C ABI with host buffers
     x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -500,42 +535,162 @@ def run_ours(args):
         e_ends[i].record(stream)
         e_ends[i].synchronize()
     e2e_ms = reduce_max(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps, dev)
-    e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
+    e2e = {"value": ctx.world * T / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": x_host.numel() * 2 + lg_host.numel() * 4,
            "d2h_bytes_per_step": out_host.numel() * 2}
 
-    # ---- CPU baseline (rank 0, one GPU)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = wl.T if wl.T <= 128 else 16
-        dt, tok, threads, _ = cpu_oracle_sample(wl, n)
-        cpu = {"value": tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": (f"all {tok} tokens of the batch" if tok == wl.T else
-                          f"first {tok} of {wl.T} tokens") +
-                         "; weights quantised by the oracle before timing"}
+    if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return 0
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(wl),
-        "roofline": dict(roof, traffic=traffic,
-                         kernel="moe_expert_mlp (grouped gate/up+SwiGLU and down GEMMs)",
-                         algorithmic_bytes=mlp_bytes, ms=mlp_ms, peak_source=peak_kind),
+    return {
+        "value": value, "ms_per_step": ms_per_step, "config": config_dict(wl),
+        "roofline": roof,
         "layer_roofline": {"bytes": layer_bytes, "flops": layer_flops,
                            "frac_of_measured": t_roof_meas / (ms_per_step / 1e3),
                            "frac_of_spec_8TBs_2.25PF": t_roof_spec / (ms_per_step / 1e3),
                            "touched_experts": touched},
-        "router": router,
-        "quantize": quant,
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": launches_per_layer(T, E, k) * args.steps,
+        "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
         "wall_s_timed_region": wall, "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),
+    }
+
+
+def unquantised_timing(moe, ctx, wl, weights, bf16_weights) -> dict:
+    """The grouped expert MLP on the workload's unquantised bf16 weights
+    (moe_expert_mlp_unquantised) beside the same call on the MXFP4 weights
+    (moe_expert_mlp), on the same permuted rows, L2 flushed before each call:
+    weight bytes streamed and time of each."""
+    import torch
+
+    dev, stream, flush, steps = ctx.dev, ctx.stream, ctx.flush, ctx.args.steps
+    D, F, E, T, k = wl.d_model, wl.d_ff, wl.E, wl.T, wl.k
+    S = T * k
+    shape = moe.make_shape(T, E, k, D, F)
+    x = torch.from_numpy(syn.activations(wl).view(np.int16)).to(dev).view(torch.bfloat16)
+    logits = torch.from_numpy(syn.logits(wl)).to(dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    tw = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    ss = torch.empty(S, dtype=torch.int32, device=dev)
+    sp = torch.empty(S, dtype=torch.int32, device=dev)
+    xp = torch.empty((S, D), dtype=torch.bfloat16, device=dev)
+    moe.moe_route(logits, k, idx, tw, stream)
+    moe.moe_permute(idx, x, shape, counts, offsets, ss, sp, xp, None, stream)
+    h = torch.empty((S, F), dtype=torch.bfloat16, device=dev)
+    yp = torch.empty((S, D), dtype=torch.bfloat16, device=dev)
+    ws_q = moe.alloc_workspace(shape, moe.WS_EXPERT_MLP, dev)
+    ws_u = moe.alloc_workspace(shape, moe.WS_EXPERT_MLP_UNQUANTISED, dev)
+    bf_gu, bf_dn = bf16_weights
+    calls = {
+        "mxfp4": lambda: moe.moe_expert_mlp(xp, offsets, shape, *weights, h, yp, ws_q, stream),
+        "bf16": lambda: moe.moe_expert_mlp_unquantised(xp, offsets, shape, bf_gu, bf_dn, h, yp,
+                                                       ws_u, stream),
+    }
+    torch.cuda.synchronize()
+    touched = int((counts > 0).sum().item())
+    out = {"call": "moe_expert_mlp_unquantised vs moe_expert_mlp", "workload": wl.name}
+    for name, call in calls.items():
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps + 2):
+            flush.fill_(i & 0xFF)
+            if i >= 2:
+                st[i - 2].record(stream)
+            call()
+            if i >= 2:
+                en[i - 2].record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in zip(st, en))
+        wbytes = touched * (expert_bytes(wl) if name == "mxfp4" else 3 * D * F * 2)
+        out[name] = {"ms": ms, "weight_bytes": wbytes,
+                     "GB/s": (wbytes + 2 * S * D * 2) / (ms / 1e3) / 1e9}
+    ws_st = (int(ws_q[:4].view(torch.int32).item()), int(ws_u[:4].view(torch.int32).item()))
+    if ws_st != (0, 0):
+        raise RuntimeError(f"expert MLP reported device status {ws_st}")
+    out["bf16_over_mxfp4_bytes"] = out["bf16"]["weight_bytes"] / out["mxfp4"]["weight_bytes"]
+    out["bf16_over_mxfp4_time"] = out["bf16"]["ms"] / out["mxfp4"]["ms"]
+    return out
+
+
+def router_timing(moe, ctx, wl):
+    """moe_router_topk on the workload's tokens against a seeded bf16 router
+    matrix [E][D], L2 flushed before each call."""
+    import torch
+
+    dev, stream, flush, steps = ctx.dev, ctx.stream, ctx.flush, ctx.args.steps
+    T, D, E, k = wl.T, wl.d_model, wl.E, wl.k
+    x = torch.from_numpy(syn.activations(wl).view(np.int16)).to(dev).view(torch.bfloat16)
+    w_router = torch.from_numpy(syn.normal_bf16(wl.seed, 40, (E, D), sigma=1.0 / D ** 0.5)
+                                .view(np.int16)).to(dev).view(torch.bfloat16)
+    r_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    r_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps + 2):
+        flush.fill_(i & 0xFF)
+        if i >= 2:
+            st[i - 2].record(stream)
+        moe.moe_router_topk(x, w_router, k, r_idx, r_w, None, None, stream)
+        if i >= 2:
+            en[i - 2].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in zip(st, en))
+    nbytes = T * D * 2 + E * D * 2 + T * k * 8
+    return {"call": "moe_router_topk", "workload": wl.name, "ms": ms, "bytes": nbytes,
+            "GB/s": nbytes / (ms / 1e3) / 1e9, "TFLOP/s": 2.0 * T * D * E / (ms / 1e3) / 1e12}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_quantised_mixture_b200 as moe
+
+    ctx = Ctx(args)
+    names = [args.workload] if args.workload else [HEADLINE] + OTHERS
+    results = {}
+    extras = {}
+    cache = {}  # weights shared by workloads of the same layer (20B decode and prefill)
+    for name in names:
+        wl = syn.WORKLOADS[name]
+        key = (wl.E, wl.d_model, wl.d_ff, wl.seed, wl.outlier_p, wl.w_sigma)
+        if key not in cache:
+            cache.clear()
+            torch.cuda.empty_cache()
+            cache[key] = quantised_weights(moe, ctx, wl, keep_first_chunk=(name == names[0]),
+                                           keep_bf16=(name == UNQUANTISED_AT))
+        weights, keep = cache[key]
+        results[name] = measure_workload(moe, ctx, wl, weights)
+        if name == UNQUANTISED_AT:
+            extras["unquantised"] = unquantised_timing(moe, ctx, wl, weights, keep["bf16"])
+            keep["bf16"] = None
+        if name == names[0]:
+            extras["router"] = router_timing(moe, ctx, wl)
+            extras["quantize"] = quantiser_timings(moe, keep["first"], ctx.flush, ctx.stream,
+                                                   args.steps, ctx.peaks[0])
+            keep["first"] = None
+        torch.cuda.empty_cache()
+    if ctx.world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if ctx.rank != 0:
+        return 0
+    head = results[names[0]]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ctx.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": head["config"],
+        "roofline": head["roofline"], "layer_roofline": head["layer_roofline"],
+        "cpu_baseline": head["cpu_baseline"], "e2e": head["e2e"], "clocks": head["clocks"],
+        "gpu_launches": head["gpu_launches"],
+        "wall_s_timed_region": head["wall_s_timed_region"],
+        "step_ms_min": head["step_ms_min"], "step_ms_max": head["step_ms_max"],
+        "router": extras.get("router"), "quantize": extras.get("quantize"),
+        "unquantised": extras.get("unquantised"),
+        "per_workload": {n: r for n, r in results.items() if n != names[0]},
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -250,6 +250,64 @@ MOE_API moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets
                           const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm,
                           void* ws, size_t ws_bytes, moe_stream stream);
 
+/* moe_expert_mlp_ex -- moe_expert_mlp with the GEMM path chosen by the
+ * caller.  Same operation, passages, arguments and errors as
+ * moe_expert_mlp; the results of the two paths agree within the layer
+ * tolerance (both take exact products of the bf16 rows and the MXFP4
+ * weights; only the fp32 accumulation order differs, and the block-scaled
+ * path drops bits of an activation more than 2^13 below its 32-block's
+ * largest, below 2^-20 of that largest).
+ *   path  MOE_MLP_PATH_AUTO: the path moe_expert_mlp takes (block-scaled
+ *         when twice the mean routed rows per expert is at most 64);
+ *         MOE_MLP_PATH_BLOCK_SCALED: tcgen05 block-scaled MMAs on the E2M1
+ *         codes, each bf16 row split exactly into two E4M3 pieces;
+ *         MOE_MLP_PATH_BF16_DECODE: the codes decoded to bf16 into tensor
+ *         memory, bf16 MMAs.  Any other value: MOE_ERR_INVALID_ARG.
+ *   ws    moe_workspace_size(shape, 1, 3 or 4) bytes for AUTO, BLOCK_SCALED
+ *         or BF16_DECODE respectively; first 4 bytes = device status word.
+ *   test_timeout_cta  testing support, -1 in normal use.  A value c >= 0
+ *         makes the first pipeline wait of the MMA issuer in CTA c of the
+ *         first GEMM give up after a short bounded wait on a barrier that
+ *         nothing completes, as a real timeout would: the device status
+ *         word becomes MOE_ERR_TIMEOUT, every CTA unwinds after draining
+ *         its own copies and MMAs, and the outputs are unspecified.  The
+ *         next call runs normally.                                        */
+#define MOE_MLP_PATH_AUTO 0
+#define MOE_MLP_PATH_BLOCK_SCALED 1
+#define MOE_MLP_PATH_BF16_DECODE 2
+MOE_API moe_status moe_expert_mlp_ex(const uint16_t* x_perm, const int32_t* offsets,
+                                     moe_shape shape, const uint8_t* wgu_q,
+                                     const uint8_t* wgu_s, const uint8_t* wdn_q,
+                                     const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm,
+                                     void* ws, size_t ws_bytes, int32_t path,
+                                     int32_t test_timeout_cta, moe_stream stream);
+
+/* moe_expert_mlp_unquantised -- the grouped SwiGLU expert MLP with
+ * unquantised bf16 expert weights: the comparison point for the MXFP4 path.
+ * Passage: "Tricks from OpenAI gpt-oss you can use with transformers"
+ * (summary), section 7, and agentlenshq (ja), "What is MXFP4" (without
+ * MXFP4 the experts are held in bf16, about four times the memory);
+ * SwiGLU experts ("Welcome GPT OSS ...", section 4).
+ * For every expert e and every permuted row r in [offsets[e], offsets[e+1]):
+ *   g = x_perm[r] . Wg_e^T, u = x_perm[r] . Wu_e^T   (fp32 accumulation of
+ *                                                    exact bf16 products)
+ *   h[r] = bf16_rne(silu(g) * u),   y_perm[r] = bf16_rne(h[r] . Wd_e^T)
+ *   x_perm  in   [S][D] bf16; offsets in [E+1] as produced by moe_permute
+ *   w_gu    in   bf16 [E][2F][D] (rows [0,F) gate, [F,2F) up)
+ *   w_dn    in   bf16 [E][D][F]
+ *   h       out  [S][F] bf16 (caller-owned intermediate)
+ *   y_perm  out  [S][D] bf16
+ *   ws      in   moe_workspace_size(shape, 5) bytes; first 4 bytes = device
+ *                status word (cleared by the call; MOE_ERR_TIMEOUT if a
+ *                bounded wait gave up)
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_WORKSPACE,
+ * MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA; device status MOE_ERR_TIMEOUT.      */
+MOE_API moe_status moe_expert_mlp_unquantised(const uint16_t* x_perm, const int32_t* offsets,
+                                              moe_shape shape, const uint16_t* w_gu,
+                                              const uint16_t* w_dn, uint16_t* h,
+                                              uint16_t* y_perm, void* ws, size_t ws_bytes,
+                                              moe_stream stream);
+
 /* moe_combine -- routing-weighted, deterministic gather-sum.
  * Passage: "Welcome GPT OSS ..." (summary), section 4 (the softmax weights
  * of the chosen experts mix their outputs).
@@ -268,7 +326,9 @@ MOE_API moe_status moe_combine(const uint16_t* y_perm, const int32_t* slot_pos,
  * in the caller's workspace (moe_workspace_size(shape, 2) bytes).
  *   x in [T][D] bf16; logits in [T][E] fp32; weights as moe_expert_mlp;
  *   out out [T][D] bf16.  The first 4 bytes of ws are the device status
- *   word; the call resets it to MOE_OK before its first kernel.
+ *   word; the call's first kernel resets it to MOE_OK.  Every check that
+ *   can refuse the call (shape, pointers, workspace, device, the GEMM
+ *   configuration and its tensor maps) is made before the first launch.
  * Errors: the union of the four calls.                                   */
 MOE_API moe_status moe_layer_forward(const uint16_t* x, const float* logits,
                              moe_shape shape, const uint8_t* wgu_q,
@@ -287,7 +347,8 @@ MOE_API moe_status moe_layer_forward(const uint16_t* x, const float* logits,
  * library, which every GPU that loads the library holds until the process
  * exits.  The first call on a device looks up that array's device address
  * (cudaGetSymbolAddress, with the device current); make that first call
- * before any stream capture.
+ * before any stream capture.  A lookup that fails (MOE_ERR_CUDA) is not
+ * remembered: the next call on that device tries again.
  *   Arguments, layouts and errors are those of moe_layer_forward, minus the
  *   workspace.  A shape with moe_workspace_size(shape, 2) above
  *   MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_WORKSPACE before
@@ -297,8 +358,9 @@ MOE_API moe_status moe_layer_forward(const uint16_t* x, const float* logits,
  *   contents: each call clears the part that must start at zero (the device
  *   status word) and overwrites the rest before reading it.  Calls that can
  *   overlap on the GPU (other streams, other threads) race on the array and
- *   must be serialised by the caller; the device status word is not
- *   readable through this entry (use moe_layer_forward when it must be).  */
+ *   must be serialised by the caller.  The layer's device status word
+ *   (MOE_ERR_TIMEOUT if a bounded wait gave up) lives in the array too:
+ *   moe_layer_static_status copies it out.                              */
 #define MOE_STATIC_SCRATCH_BYTES (16u << 20)
 MOE_API moe_status moe_layer_forward_static(const uint16_t* x, const float* logits,
                                             moe_shape shape, const uint8_t* wgu_q,
@@ -306,8 +368,19 @@ MOE_API moe_status moe_layer_forward_static(const uint16_t* x, const float* logi
                                             const uint8_t* wdn_s, uint16_t* out,
                                             moe_stream stream);
 
+/* moe_layer_static_status -- the device status word of the last
+ * moe_layer_forward_static call on the current device, copied on `stream`
+ * (one 4-byte device-to-device copy, no allocation) into d_status, a
+ * caller-owned, 4-byte aligned device int32; read it after the stream
+ * syncs.  Like the entry it serves, it has no counterpart in the pages.
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.        */
+MOE_API moe_status moe_layer_static_status(int32_t* d_status, moe_stream stream);
+
 /* moe_workspace_size -- bytes of device workspace a call needs.
- * which: 0 = moe_permute, 1 = moe_expert_mlp, 2 = moe_layer_forward.
+ * which: 0 = moe_permute, 1 = moe_expert_mlp, 2 = moe_layer_forward,
+ * 3 = moe_expert_mlp_ex with MOE_MLP_PATH_BLOCK_SCALED,
+ * 4 = moe_expert_mlp_ex with MOE_MLP_PATH_BF16_DECODE,
+ * 5 = moe_expert_mlp_unquantised.
  * Returns 0 for an unsupported shape or an unknown `which`.  Host only.  */
 MOE_API size_t moe_workspace_size(moe_shape shape, int which);
 

@@ -25,6 +25,13 @@ MOE_ERR_NONFINITE = 6
 MOE_ERR_TIMEOUT = 7
 
 WS_PERMUTE, WS_EXPERT_MLP, WS_LAYER = 0, 1, 2
+WS_EXPERT_MLP_BLOCK_SCALED, WS_EXPERT_MLP_BF16_DECODE = 3, 4
+WS_EXPERT_MLP_UNQUANTISED = 5
+
+# GEMM path of moe_expert_mlp_ex
+MOE_MLP_PATH_AUTO = 0
+MOE_MLP_PATH_BLOCK_SCALED = 1  # tcgen05 block-scaled MMA on the E2M1 codes
+MOE_MLP_PATH_BF16_DECODE = 2   # codes decoded to bf16 into tensor memory
 
 MOE_QUANT_RHT = 1  # random-sign Hadamard transform of each 32-block along K
 MOE_QUANT_SR = 2   # stochastic rounding
@@ -65,12 +72,19 @@ def _load() -> ctypes.CDLL:
     lib.moe_permute.restype = st
     lib.moe_expert_mlp.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_expert_mlp.restype = st
+    lib.moe_expert_mlp_ex.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp, vp, sz, i32, i32,
+                                      vp]
+    lib.moe_expert_mlp_ex.restype = st
+    lib.moe_expert_mlp_unquantised.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_expert_mlp_unquantised.restype = st
     lib.moe_combine.argtypes = [vp, vp, vp, moe_shape, vp, vp]
     lib.moe_combine.restype = st
     lib.moe_layer_forward.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_layer_forward.restype = st
     lib.moe_layer_forward_static.argtypes = [vp, vp, moe_shape, vp, vp, vp, vp, vp, vp]
     lib.moe_layer_forward_static.restype = st
+    lib.moe_layer_static_status.argtypes = [vp, vp]
+    lib.moe_layer_static_status.restype = st
     lib.moe_workspace_size.argtypes = [moe_shape, ctypes.c_int]
     lib.moe_workspace_size.restype = sz
     lib.moe_status_string.argtypes = [st]
@@ -178,6 +192,27 @@ def moe_expert_mlp(x_perm, offsets, shape: moe_shape, wgu_q, wgu_s, wdn_q, wdn_s
                                                 _p(ws), _nbytes(ws), _s(stream)))
 
 
+def moe_expert_mlp_ex(x_perm, offsets, shape: moe_shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm, ws,
+                      path: int = MOE_MLP_PATH_AUTO, test_timeout_cta: int = -1,
+                      stream=None) -> None:
+    """moe_expert_mlp on a chosen GEMM path (MOE_MLP_PATH_*); ws sized by
+    moe_workspace_size(shape, WS_EXPERT_MLP / _BLOCK_SCALED / _BF16_DECODE).
+    test_timeout_cta >= 0 is testing support (see the C header)."""
+    _check("moe_expert_mlp_ex",
+           lib.moe_expert_mlp_ex(_p(x_perm), _p(offsets), shape, _p(wgu_q), _p(wgu_s), _p(wdn_q),
+                                 _p(wdn_s), _p(h), _p(y_perm), _p(ws), _nbytes(ws), int(path),
+                                 int(test_timeout_cta), _s(stream)))
+
+
+def moe_expert_mlp_unquantised(x_perm, offsets, shape: moe_shape, w_gu, w_dn, h, y_perm, ws,
+                               stream=None) -> None:
+    """The grouped expert MLP on unquantised bf16 weights w_gu [E][2F][D] and
+    w_dn [E][D][F]; ws sized by moe_workspace_size(shape, WS_EXPERT_MLP_UNQUANTISED)."""
+    _check("moe_expert_mlp_unquantised",
+           lib.moe_expert_mlp_unquantised(_p(x_perm), _p(offsets), shape, _p(w_gu), _p(w_dn),
+                                          _p(h), _p(y_perm), _p(ws), _nbytes(ws), _s(stream)))
+
+
 def moe_combine(y_perm, slot_pos, topk_w, shape: moe_shape, out, stream=None) -> None:
     _check("moe_combine", lib.moe_combine(_p(y_perm), _p(slot_pos), _p(topk_w), shape, _p(out),
                                           _s(stream)))
@@ -202,6 +237,12 @@ def moe_layer_forward_static(x, logits, shape: moe_shape, wgu_q, wgu_s, wdn_q, w
                                         _p(wdn_s), _p(out), _s(stream)))
 
 
+def moe_layer_static_status(d_status, stream=None) -> None:
+    """Copy the device status word of the last moe_layer_forward_static call
+    on this device into d_status (a device int32 tensor), on the stream."""
+    _check("moe_layer_static_status", lib.moe_layer_static_status(_p(d_status), _s(stream)))
+
+
 def alloc_workspace(shape: moe_shape, which: int, device="cuda"):
     """A device byte tensor of moe_workspace_size(shape, which) bytes (at least 256)."""
     import torch
@@ -213,6 +254,7 @@ def alloc_workspace(shape: moe_shape, which: int, device="cuda"):
 __all__ = ["moe_shape", "make_shape", "MoeError", "mxfp4_quantize", "mxfp4_quantize_sr_rht",
            "MOE_QUANT_RHT", "MOE_QUANT_SR", "moe_route",
            "moe_router_topk", "moe_permute",
-           "moe_expert_mlp", "moe_combine", "moe_layer_forward", "moe_layer_forward_static",
+           "moe_expert_mlp", "moe_expert_mlp_ex", "moe_expert_mlp_unquantised", "moe_combine", "moe_layer_forward",
+           "moe_layer_forward_static", "moe_layer_static_status",
            "moe_workspace_size",
            "moe_status_string", "alloc_workspace", "lib", "LIB_PATH"]

@@ -9,21 +9,22 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "mlp_plan.cuh"
 
 namespace moe {
 
 moe_status route_launch(const float* logits, int T, int E, int k, int32_t* idx, float* w,
-                        cudaStream_t stream);
+                        int32_t* clear_status, cudaStream_t stream);
 moe_status permute_launch(const int32_t* idx, const uint16_t* x, const moe_shape& sh,
                           int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
-                          int32_t* slot_pos, uint16_t* x_perm, cudaStream_t stream);
-size_t expert_mlp_workspace(const moe_shape& sh);
-moe_status expert_mlp_launch(const uint16_t* x_perm, const int32_t* offsets, const moe_shape& sh,
-                             const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
-                             const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
-                             int32_t* status, cudaStream_t stream);
+                          int32_t* slot_pos, uint16_t* x_perm, int NT, Tile* tiles,
+                          int* n_tiles, cudaStream_t stream);
 moe_status combine_launch(const uint16_t* y_perm, const int32_t* slot_pos, const float* w,
                           const moe_shape& sh, uint16_t* out, cudaStream_t stream);
+size_t unquantised_workspace(const moe_shape& sh);
+moe_status unquantised_mlp(const uint16_t* x_perm, const int32_t* offsets, const moe_shape& sh,
+                           const uint16_t* w_gu, const uint16_t* w_dn, uint16_t* h,
+                           uint16_t* y_perm, void* ws, int32_t* status, cudaStream_t stream);
 
 namespace {
 
@@ -78,7 +79,7 @@ LayerWs layer_ws(const moe_shape& s) {
   L.x_perm = take(S * s.d_model * 2);
   L.h = take(S * s.d_ff * 2);
   L.y_perm = take(S * s.d_model * 2);
-  L.mlp = take(expert_mlp_workspace(s));
+  L.mlp = take(expert_mlp_workspace(s, kPathAuto));
   L.total = o;
   return L;
 }
@@ -124,9 +125,15 @@ size_t moe_workspace_size(moe_shape shape, int which) {
     case 0:
       return 0;
     case 1:
-      return kMlpStatusBytes + expert_mlp_workspace(shape);
+      return kMlpStatusBytes + expert_mlp_workspace(shape, kPathAuto);
     case 2:
       return layer_ws(shape).total;
+    case 3:
+      return kMlpStatusBytes + expert_mlp_workspace(shape, kPathBlockScaled);
+    case 4:
+      return kMlpStatusBytes + expert_mlp_workspace(shape, kPathBf16Decode);
+    case 5:
+      return kMlpStatusBytes + unquantised_workspace(shape);
     default:
       return 0;
   }
@@ -154,12 +161,15 @@ const char* moe_status_string(moe_status status) {
   return "MOE_ERR_UNKNOWN";
 }
 
-moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, moe_shape shape,
-                          const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
-                          const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
-                          size_t ws_bytes, moe_stream stream) {
+moe_status moe_expert_mlp_ex(const uint16_t* x_perm, const int32_t* offsets, moe_shape shape,
+                             const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
+                             const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
+                             size_t ws_bytes, int32_t path, int32_t test_timeout_cta,
+                             moe_stream stream) {
   using namespace moe;
   if (!shape_ok(shape)) return MOE_ERR_SHAPE;
+  if (path != kPathAuto && path != kPathBlockScaled && path != kPathBf16Decode)
+    return MOE_ERR_INVALID_ARG;
   if (shape.T == 0) return MOE_OK;
   const void* ptrs[] = {x_perm, offsets, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm};
   for (const void* p : ptrs)
@@ -167,17 +177,49 @@ moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, moe_sh
   if (!aligned32(wgu_q) || !aligned32(wdn_q)) return MOE_ERR_INVALID_ARG;
   // the first kMlpStatusBytes of ws hold the device status word, the rest
   // is the GEMMs' workspace (same alignment class as ws itself)
-  const size_t need = kMlpStatusBytes + expert_mlp_workspace(shape);
+  const size_t need = kMlpStatusBytes + expert_mlp_workspace(shape, path);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   moe_status st = check_device();
   if (st != MOE_OK) return st;
+  MlpPlan plan;
+  if ((st = expert_mlp_plan(shape, path, x_perm, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm,
+                            static_cast<char*>(ws) + kMlpStatusBytes, &plan)) != MOE_OK)
+    return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  return expert_mlp_launch(x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm,
-                           static_cast<char*>(ws) + kMlpStatusBytes, static_cast<int32_t*>(ws), s);
+  MlpInput in{};
+  in.offsets = offsets;
+  return expert_mlp_enqueue(plan, in, static_cast<int32_t*>(ws), test_timeout_cta < 0 ? -1 : test_timeout_cta, s);
+}
+
+moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, moe_shape shape,
+                          const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
+                          const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
+                          size_t ws_bytes, moe_stream stream) {
+  return moe_expert_mlp_ex(x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm, ws,
+                           ws_bytes, MOE_MLP_PATH_AUTO, -1, stream);
+}
+
+moe_status moe_expert_mlp_unquantised(const uint16_t* x_perm, const int32_t* offsets,
+                                      moe_shape shape, const uint16_t* w_gu, const uint16_t* w_dn,
+                                      uint16_t* h, uint16_t* y_perm, void* ws, size_t ws_bytes,
+                                      moe_stream stream) {
+  using namespace moe;
+  if (!shape_ok(shape)) return MOE_ERR_SHAPE;
+  if (shape.T == 0) return MOE_OK;
+  const void* ptrs[] = {x_perm, offsets, w_gu, w_dn, h, y_perm};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const size_t need = kMlpStatusBytes + unquantised_workspace(shape);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  moe_status st = check_device();
+  if (st != MOE_OK) return st;
+  return unquantised_mlp(x_perm, offsets, shape, w_gu, w_dn, h, y_perm,
+                         static_cast<char*>(ws) + kMlpStatusBytes, static_cast<int32_t*>(ws),
+                         static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape shape,
@@ -198,10 +240,7 @@ moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(ws);
   auto at = [&](size_t off) { return static_cast<void*>(base + off); };
-  if (cudaMemsetAsync(at(L.status), 0, 4, s) != cudaSuccess) {
-    cudaGetLastError();
-    return MOE_ERR_CUDA;
-  }
+  int32_t* status = static_cast<int32_t*>(at(L.status));
   int32_t* idx = static_cast<int32_t*>(at(L.idx));
   float* w = static_cast<float*>(at(L.w));
   int32_t* counts = static_cast<int32_t*>(at(L.counts));
@@ -211,13 +250,31 @@ moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape s
   uint16_t* x_perm = static_cast<uint16_t*>(at(L.x_perm));
   uint16_t* h = static_cast<uint16_t*>(at(L.h));
   uint16_t* y_perm = static_cast<uint16_t*>(at(L.y_perm));
-  if ((st = route_launch(logits, shape.T, shape.E, shape.k, idx, w, s)) != MOE_OK) return st;
-  if ((st = permute_launch(idx, x, shape, counts, offsets, sorted_slot, slot_pos, x_perm, s)) !=
+  // everything that can refuse the call happens here, before the first launch
+  MlpPlan plan;
+  const bool block_scaled = resolve_path(shape, kPathAuto) == kPathBlockScaled;
+  if ((st = expert_mlp_plan(shape, kPathAuto, x_perm, wgu_q, wgu_s, wdn_q, wdn_s,
+                            block_scaled ? nullptr : h, y_perm, at(L.mlp), &plan)) != MOE_OK)
+    return st;
+  const int NT = mlp_tile_width(shape, kPathAuto);
+  // route (its first thread also clears the status word), then permute with
+  // the GEMMs' tile list; the block-scaled path splits its rows straight from
+  // x, so only the other path gathers x_perm
+  if ((st = route_launch(logits, shape.T, shape.E, shape.k, idx, w, status, s)) != MOE_OK)
+    return st;
+  if ((st = permute_launch(idx, x, shape, counts, offsets, sorted_slot, slot_pos,
+                           block_scaled ? nullptr : x_perm, NT, plan.tiles, plan.n_tiles, s)) !=
       MOE_OK)
     return st;
-  if ((st = expert_mlp_launch(x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm,
-                              at(L.mlp), static_cast<int32_t*>(at(L.status)), s)) != MOE_OK)
-    return st;
+  MlpInput in{};
+  in.offsets = offsets;
+  in.tiles_ready = true;
+  if (block_scaled) {
+    in.x = x;
+    in.sorted_slot = sorted_slot;
+    in.k = shape.k;
+  }
+  if ((st = expert_mlp_enqueue(plan, in, status, -1, s)) != MOE_OK) return st;
   return combine_launch(y_perm, slot_pos, w, shape, out, s);
 }
 

@@ -31,13 +31,20 @@
 // The epilogue adds rows 2t and 2t + 1 (neighbouring lanes).
 //   * gate/up: the 128 rows are 64 gate rows and the matching 64 up rows,
 //     interleaved by the copy's box order (row 2j = gate j, 2j + 1 = up j), so
-//     a lane holds both halves of SwiGLU; output h [S][F] bf16.
+//     a lane holds both halves of SwiGLU.  The epilogue rounds h to bf16
+//     (stored to h [S][F] when asked) and splits it at once into the pieces
+//     the down GEMM reads: each epilogue warp holds one whole 32-feature block
+//     of h for its tokens.
 //   * down: 128 rows of the [D][F] matrix; output y_perm [S][D] bf16.
 // The kernel is persistent: one CTA per SM walks the work items (token tile,
 // weight slice) b, b + grid, ...; its copy ring (up to 12 stages of two
 // 128-K windows each, so one barrier round trip covers 256 of K) runs on
 // across items, the weight-scale block of an item is double-buffered and so
 // is the accumulator, so one item's epilogue overlaps the next item's MMAs.
+// When an item starts, the producer asks L2 to prefetch the CTA's next
+// item's weight rows (contiguous ranges of the codes), so the ring's copies
+// of that item meet L2 rather than HBM latency while the prefetch keeps more
+// bytes in flight than the ring's shared memory could.
 // Warp roles (14 warps):
 //   warp 0      producer: per item the weight-scale bytes and the token-scale
 //               words (bulk copies), per 128-K window the weight codes (TMA,
@@ -56,14 +63,23 @@
 // The token pieces sit in a tile-padded layout (tile t owns piece rows
 // [2 t NT, 2 t NT + 2 NT)), so every copy of a tile's rows is aligned and
 // whole; the MMA's 128-row view of a stage narrower than 128 rows reads on
-// into the following shared memory, and those accumulator rows are ignored.
+// into the following shared memory, and those accumulator rows are ignored
+// (an accumulator row depends only on its own operand row and scales, so
+// whatever the padding rows hold never reaches a real token's output).
 // Every wait is bounded (2 s); on expiry the kernel records MOE_ERR_TIMEOUT
-// in the status word, drains its copies and MMAs and returns.
+// in the status word and unwinds: every role leaves its loop, the scale
+// writers complete the stage arrivals they skipped (the producer's copy
+// barrier also counts them), the producer waits for every copy it issued to
+// land and the MMA thread's last commit for every MMA it issued, and only
+// then is tensor memory freed and the CTA gone.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <atomic>
+
 #include "common.cuh"
+#include "mlp_plan.cuh"
 #include "tc_sm100.cuh"
 
 namespace moe {
@@ -81,10 +97,8 @@ constexpr int kMaxStages = 12;      // copy ring depth limit (stage slot s also 
 constexpr int kSlotCols = 8 * WPS;  // per stage and window: 4 token-scale + 4 weight-scale columns
 constexpr int kTmemCols = 512;      // two accumulators of BN columns, then the scale slots
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
-struct Tile {
-  int e, row0, nrows, pad;
-};
+constexpr uint64_t kTestWaitNs = 200000ull;  // the injected wait of test_timeout_cta
+constexpr uint32_t kPrefetchChunk = 32768;   // bytes per L2 prefetch instruction
 
 // Per work item the producer also loads an auxiliary block: the weight-scale
 // bytes of the item's rows [BN][K/32] and the token-scale words of its tile
@@ -110,6 +124,35 @@ __host__ __device__ inline SmemLayout smem_layout(int NT, int NS, int NB, int K)
 __host__ __device__ __forceinline__ int stage_k0(int st, int K) {
   return st * BKS < K - BKS ? st * BKS : K - BKS;
 }
+
+// ------------------------------------------------ exact two-piece E4M3 split
+
+// Block exponent t = floor(log2 amax) - 7 from the biased exponent field;
+// zero and subnormal blocks take the floor -123, which keeps both scale
+// bytes (t + 127 for hi, t + 123 for lo) >= 0.
+__device__ __forceinline__ int split_exponent(float amax) {
+  const int ebits = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+  return max(ebits - 127 - 7, -123);
+}
+
+// Four bf16-exact values of one block -> their hi and lo E4M3 bytes.
+__device__ __forceinline__ void split4(const float (&v)[4], int t, uint32_t& hi4, uint32_t& lo4) {
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - t) << 23);  // 2^-t
+  hi4 = 0;
+  lo4 = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float u = v[j] * inv;
+    const __nv_fp8_storage_t h8 = __nv_cvt_float_to_fp8(u, __NV_SATFINITE, __NV_E4M3);
+    const float hf = __half2float(__half(__nv_cvt_fp8_to_halfraw(h8, __NV_E4M3)));
+    const __nv_fp8_storage_t l8 =
+        __nv_cvt_float_to_fp8((u - hf) * 16.0f, __NV_SATFINITE, __NV_E4M3);
+    hi4 |= static_cast<uint32_t>(h8) << (8 * j);
+    lo4 |= static_cast<uint32_t>(l8) << (8 * j);
+  }
+}
+
+// ------------------------------------------------------------------ waits
 
 __device__ __forceinline__ void abort_cta(volatile int* abort, int32_t* status) {
   *abort = 1;
@@ -143,20 +186,63 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return r;
 }
 
+// Ask L2 for the weight rows of work item i: gate/up, rows [f0, f0 + 64) of
+// the gate and of the up half (two contiguous ranges); down, rows
+// [d0, d0 + 128) (one range); both clipped to the matrix.
+template <bool GATE_UP>
+__device__ __forceinline__ void prefetch_item(const uint8_t* wq, const Tile* tiles, int i,
+                                              int n_mt, int rows_per_expert, int K) {
+  const int t = i / n_mt, mt = i % n_mt;
+  const int e = __ldg(&tiles[t].e);
+  const int64_t row_bytes = K / 2;
+  const uint8_t* base = wq + static_cast<int64_t>(e) * rows_per_expert * row_bytes;
+  auto range = [&](int64_t r0, int rows) {
+    const uint8_t* p = base + r0 * row_bytes;
+    const uint32_t bytes = static_cast<uint32_t>(rows * row_bytes);
+    for (uint32_t o = 0; o < bytes; o += kPrefetchChunk)
+      tc::prefetch_l2(p + o, min(kPrefetchChunk, bytes - o));
+  };
+  if (GATE_UP) {
+    const int F = rows_per_expert / 2, f0 = mt * (BN / 2);
+    const int rows = min(BN / 2, F - f0);
+    range(f0, rows);
+    range(F + f0, rows);
+  } else {
+    const int d0 = mt * BN;
+    range(d0, min(BN, rows_per_expert - d0));
+  }
+}
+
+// Arguments of one GEMM launch.
+struct GemmArgs {
+  const uint32_t* sfx_words;  // token-scale words of the input pieces
+  const uint8_t* scales;      // weight scale bytes [E][R][K/32]
+  const uint8_t* wq;          // weight codes [E][R][K/2] (for the L2 prefetch)
+  const Tile* tiles;
+  const int* n_tiles;
+  int rows_per_expert, K, NS, NB, out_ld;
+  uint16_t* out;  // h (gate/up; may be null) or y_perm (down)
+  // gate/up only: the pieces of h for the down GEMM, [2 * padded rows][F]
+  // bytes, and their scale words [tiles][F/128 windows][2 NT]
+  uint8_t* pieces_out;
+  uint32_t* words_out;
+  int32_t* status;
+  int fail_cta;
+};
+
 template <int NT, bool GATE_UP>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_mx_gemm(const __grid_constant__ CUtensorMap map_w,
                     const __grid_constant__ CUtensorMap map_w_tail,
-                    const __grid_constant__ CUtensorMap map_x,
-                    const uint32_t* __restrict__ sfx_words, const uint8_t* __restrict__ scales,
-                    const Tile* __restrict__ tiles, const int* __restrict__ n_tiles_dev,
-                    int rows_per_expert, int K, int NS, int NB, int out_ld,
-                    uint16_t* __restrict__ out, int32_t* __restrict__ status) {
+                    const __grid_constant__ CUtensorMap map_x, const GemmArgs args) {
   constexpr int XR = 2 * NT;  // token piece rows per window
   constexpr uint32_t X_BYTES = XR * BKS;
   constexpr uint32_t IDESC = tc::idesc_mx(tc::kFmtE4M3, tc::kFmtE2M1, MM, BN);
   static_assert(XR <= MM && (X_BYTES % 1024) == 0, "token tile of 8..64 tokens");
-  const int n_tiles = __ldg(n_tiles_dev);
+  const int rows_per_expert = args.rows_per_expert, K = args.K, NS = args.NS, NB = args.NB;
+  const Tile* __restrict__ tiles = args.tiles;
+  int32_t* status = args.status;
+  const int n_tiles = __ldg(args.n_tiles);
   const int F = rows_per_expert / 2;
   const int n_mt = GATE_UP ? (F + BN / 2 - 1) / (BN / 2) : (rows_per_expert + BN - 1) / BN;
   const int n_items = n_tiles * n_mt;
@@ -177,8 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* dfull = sfree + 2;            // [2] accumulator complete
   uint64_t* dempty = dfull + 2;           // [2] accumulator read by the epilogue
   uint64_t* drain = dempty + 2;           // every MMA issued has completed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* never = drain + 1;            // completed by nothing (the injected test wait)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* prod_stages = abort_flag + 1;  // stages the producer issued (read on unwind)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwin = (K + BKS - 1) / BKS;    // 128-K windows
@@ -199,7 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&dempty[a], kEpiWarps);
     }
     tc::mbar_init(drain, 1);
+    tc::mbar_init(never, 1);
     *abort_flag = 0;
+    *prod_stages = 0;
     tc::fence_mbar_init();
     tc::tma_prefetch_desc(&map_w);
     tc::tma_prefetch_desc(&map_w_tail);
@@ -214,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t t_sf = tmem + 2 * BN;  // stage slot s: columns t_sf + s * kSlotCols ...
+  int my_stages = 0;  // scale writers: stages this warp has arrived on
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -225,6 +316,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
         const int t = i / n_mt, mt = i % n_mt;
         const Tile tile = tiles[t];
+        // this item's rows were prefetched with the previous item (the first
+        // item's now); ask for the next item's
+        if (it == 0) prefetch_item<GATE_UP>(args.wq, tiles, i, n_mt, rows_per_expert, K);
+        if (i + static_cast<int>(gridDim.x) < n_items)
+          prefetch_item<GATE_UP>(args.wq, tiles, i + gridDim.x, n_mt, rows_per_expert, K);
         const int b = it % NB, use = it / NB;
         // the auxiliary buffer is free once the scale writers are done with its last item
         if (use > 0 && !wait1(&sfree[b], (use - 1) & 1, abort_flag, status)) break;
@@ -235,17 +331,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int f0 = mt * (BN / 2);
           const uint32_t bytes = static_cast<uint32_t>(min(BN / 2, F - f0)) * kscale;
           tc::mbar_arrive_expect_tx(&sbar[b], 2 * bytes + wbytes);
-          tc::bulk_load(sdst, scales + (erow + f0) * kscale, bytes, &sbar[b]);
-          tc::bulk_load(sdst + (BN / 2) * kscale, scales + (erow + F + f0) * kscale, bytes,
+          tc::bulk_load(sdst, args.scales + (erow + f0) * kscale, bytes, &sbar[b]);
+          tc::bulk_load(sdst + (BN / 2) * kscale, args.scales + (erow + F + f0) * kscale, bytes,
                         &sbar[b]);
         } else {
           const int d0 = mt * BN;
           const uint32_t bytes = static_cast<uint32_t>(min(BN, rows_per_expert - d0)) * kscale;
           tc::mbar_arrive_expect_tx(&sbar[b], bytes + wbytes);
-          tc::bulk_load(sdst, scales + (erow + d0) * kscale, bytes, &sbar[b]);
+          tc::bulk_load(sdst, args.scales + (erow + d0) * kscale, bytes, &sbar[b]);
         }
-        tc::bulk_load(sdst + L.wsc_bytes, sfx_words + static_cast<int64_t>(t) * nwin * XR, wbytes,
-                      &sbar[b]);
+        tc::bulk_load(sdst + L.wsc_bytes, args.sfx_words + static_cast<int64_t>(t) * nwin * XR,
+                      wbytes, &sbar[b]);
         const int wrow = GATE_UP ? mt * (BN / 2) : mt * BN;
         for (int st = 0; st < nstg; ++st, ++g) {
           if (g >= NS && !wait1(&empty[s_slot], s_phase ^ 1u, abort_flag, status)) {
@@ -278,11 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // drain: every copy this thread issued has landed before the CTA exits
-      for (int gg = max(0, g - NS); gg < g; ++gg)
-        tc::mbar_wait(&full[gg % NS], (gg / NS) & 1, abort_flag, kWaitLimitNs / 8);
-      for (int j = max(0, it - NB); j < it; ++j)
-        tc::mbar_wait(&sbar[j % NB], (j / NB) & 1, abort_flag, kWaitLimitNs / 8);
+      *prod_stages = g;
+      // the items whose auxiliary copies were issued: [it - NB, it) at most
+      // (their drain comes after the scale writers' catch-up, below)
+      my_stages = it;
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
@@ -297,6 +392,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t xdesc0 = tc::smem_desc_sw128(tc::smem_u32(xs));
       const uint64_t wdesc0 = tc::smem_desc_sw128(tc::smem_u32(wsm));
       const int tail_w = (K % BKS) ? nwin - 1 : nwin;  // the re-read window, if any
+      // testing only: the first wait of this CTA waits on a barrier that
+      // nothing completes, with a short limit, and gives up as a timeout would
+      if (static_cast<int>(blockIdx.x) == args.fail_cta &&
+          !tc::mbar_wait(never, 0, abort_flag, kTestWaitNs)) {
+        abort_cta(abort_flag, status);
+        ok = false;
+      }
       for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
         const uint32_t d = tmem + (it & 1) * BN;
         // accumulator it & 1 was last used by item it - 2
@@ -430,6 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the item's auxiliary block is no longer read
       if (lane == 0) tc::mbar_arrive(&sfree[b]);
     }
+    my_stages = g;
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                // tensor-memory lane quarter
@@ -447,12 +550,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
       if (16 * q < tile.nrows) {  // this quarter holds at least one real token
         const bool live_row = tl < tile.nrows;
-        uint16_t* orow = out + static_cast<int64_t>(tile.row0 + tl) * out_ld;
         const uint32_t dcol = tmem + a * BN + 64 * half;
-        // 16 accumulator columns starting at item column cc -> outputs
-        auto finish16 = [&](const uint32_t(&r)[16], int cc) {
-          // the hi lane finishes columns cc..cc+7, the lo lane cc+8..cc+15
-          float sum[8];
+        // 16 accumulator columns starting at item column cc: the hi lane
+        // finishes columns cc..cc+7, the lo lane cc+8..cc+15
+        auto sums16 = [&](const uint32_t(&r)[16], float(&sum)[8]) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float x = __uint_as_float(r[j]);
@@ -460,38 +561,104 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float recv = __shfl_xor_sync(0xFFFFFFFFu, lo ? x : y, 1);
             sum[j] = (lo ? y : x) + recv;
           }
-          const int c0 = cc + (lo ? 8 : 0);
-          if (GATE_UP) {
-            // columns 2j (gate) and 2j + 1 (up) of feature mt * 64 + j
-            const int f = mt * (BN / 2) + c0 / 2;
-            uint32_t hw[2];
+        };
+        if (GATE_UP) {
+          // This warp's 64 columns are the gate/up pairs of one 32-feature
+          // block of h, fb = mt * 64 + 32 * half; the token's two lanes hold
+          // 16 features each: group gi of this lane is features
+          // fb + 8 gi + (lo ? 4 : 0) + 0..3.
+          const int fb = mt * (BN / 2) + 32 * half;
+          float hv[16];
+          uint32_t hb[8];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              float hv[2];
+          for (int c = 0; c < 64; c += 32) {
+            uint32_t ra[16], rb[16];
+            tc::tmem_ld16(dcol + lane_base + c, ra);
+            tc::tmem_ld16(dcol + lane_base + c + 16, rb);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              float sum[8];
+              sums16(h2 ? rb : ra, sum);
+              const int gi = (c >> 4) + h2;
 #pragma unroll
               for (int p2 = 0; p2 < 2; ++p2) {
-                const float gv = sum[4 * j + 2 * p2], uv = sum[4 * j + 2 * p2 + 1];
-                hv[p2] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+                float hh[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  const float gv = sum[4 * p2 + 2 * u], uv = sum[4 * p2 + 2 * u + 1];
+                  hh[u] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+                }
+                const uint32_t w2 = pack_bf16x2(hh[0], hh[1]);
+                hb[2 * gi + p2] = w2;
+                hv[4 * gi + 2 * p2] = __uint_as_float(w2 << 16);
+                hv[4 * gi + 2 * p2 + 1] = __uint_as_float(w2 & 0xFFFF0000u);
               }
-              hw[j] = pack_bf16x2(hv[0], hv[1]);
             }
-            if (live_row && f < F) *reinterpret_cast<uint2*>(orow + f) = make_uint2(hw[0], hw[1]);
-          } else {
-            const int dd = mt * BN + c0;
-            if (live_row && dd < rows_per_expert)
-              *reinterpret_cast<uint4*>(orow + dd) =
-                  make_uint4(pack_bf16x2(sum[0], sum[1]), pack_bf16x2(sum[2], sum[3]),
-                             pack_bf16x2(sum[4], sum[5]), pack_bf16x2(sum[6], sum[7]));
           }
-        };
+          uint16_t* orow = args.out ? args.out + static_cast<int64_t>(tile.row0 + tl) * args.out_ld
+                                    : nullptr;
+          if (orow && live_row) {
+#pragma unroll
+            for (int gi = 0; gi < 4; ++gi) {
+              const int f = fb + 8 * gi + (lo ? 4 : 0);
+              if (f < F) *reinterpret_cast<uint2*>(orow + f) = make_uint2(hb[2 * gi], hb[2 * gi + 1]);
+            }
+          }
+          // the split of h for the down GEMM: the block's exponent from the
+          // token's 32 features (this lane's 16 and its neighbour's)
+          float amax = 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(hv[j]));
+          amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+          const int te = split_exponent(amax);
+          const int64_t p = static_cast<int64_t>(t) * NT + tl;  // padded row of this token
+          uint8_t* prow_hi = args.pieces_out + (2 * p) * F;
+          uint8_t* prow_lo = prow_hi + F;
+#pragma unroll
+          for (int gi = 0; gi < 4; ++gi) {
+            const float v4[4] = {hv[4 * gi], hv[4 * gi + 1], hv[4 * gi + 2], hv[4 * gi + 3]};
+            uint32_t hi4, lo4;
+            split4(v4, te, hi4, lo4);
+            const int f = fb + 8 * gi + (lo ? 4 : 0);
+            *reinterpret_cast<uint32_t*>(prow_hi + f) = hi4;
+            *reinterpret_cast<uint32_t*>(prow_lo + f) = lo4;
+          }
+          if (!lo) {
+            // scale bytes of block fb / 32 in the words of the window(s)
+            // that cover it: window b / 4 (byte b % 4), and, when F is not a
+            // multiple of 128, the moved-back last window [F - 128, F)
+            const int nwo = (F + BKS - 1) / BKS;
+            const int blk = fb / 32;
+            const int tail0 = (F % BKS) ? (F - BKS) / 32 : 0x7FFFFFFF;
+            auto put = [&](int w, int byte) {
+              uint8_t* wb = reinterpret_cast<uint8_t*>(
+                  args.words_out + (static_cast<int64_t>(t) * nwo + w) * (2 * NT) + 2 * tl);
+              wb[byte] = static_cast<uint8_t>(te + 127);
+              wb[4 + byte] = static_cast<uint8_t>(te + 123);
+            };
+            if (F % BKS == 0 || blk / 4 < nwo - 1) put(blk / 4, blk % 4);
+            if (blk >= tail0) put(nwo - 1, blk - tail0);
+          }
+        } else {
+          uint16_t* orow = args.out + static_cast<int64_t>(tile.row0 + tl) * args.out_ld;
 #pragma unroll 1
-        for (int c = 0; c < 64; c += 32) {
-          uint32_t ra[16], rb[16];
-          tc::tmem_ld16(dcol + lane_base + c, ra);
-          tc::tmem_ld16(dcol + lane_base + c + 16, rb);
-          tc::tmem_ld_wait();
-          finish16(ra, 64 * half + c);
-          finish16(rb, 64 * half + c + 16);
+          for (int c = 0; c < 64; c += 32) {
+            uint32_t ra[16], rb[16];
+            tc::tmem_ld16(dcol + lane_base + c, ra);
+            tc::tmem_ld16(dcol + lane_base + c + 16, rb);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              float sum[8];
+              sums16(h2 ? rb : ra, sum);
+              const int dd = mt * BN + 64 * half + c + 16 * h2 + (lo ? 8 : 0);
+              if (live_row && dd < rows_per_expert)
+                *reinterpret_cast<uint4*>(orow + dd) =
+                    make_uint4(pack_bf16x2(sum[0], sum[1]), pack_bf16x2(sum[2], sum[3]),
+                               pack_bf16x2(sum[4], sum[5]), pack_bf16x2(sum[6], sum[7]));
+            }
+          }
         }
       }
       // this warp has read its part of the accumulator
@@ -501,45 +668,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // ---------------------------------------------------------------- unwind
   tc::tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // A stage's copy barrier also counts the four scale writers: a writer
+    // that gave up adds the arrivals it skipped for the stages the producer
+    // issued, so those phases complete as soon as their copies land.
+    if (warp >= 2 && warp < 6 && lane == 0) {
+      const int g_p = *prod_stages;
+      for (int gg = my_stages; gg < g_p; ++gg) tc::mbar_arrive(&full[gg % NS]);
+    }
+    __syncthreads();
+  }
+  if (warp == 0 && lane == 0) {
+    // every copy this thread issued has landed before the CTA exits
+    const int g = *prod_stages, it = my_stages;
+    for (int gg = max(0, g - NS); gg < g; ++gg)
+      tc::mbar_drain(&full[gg % NS], (gg / NS) & 1, kWaitLimitNs / 8);
+    for (int j = max(0, it - NB); j < it; ++j)
+      tc::mbar_drain(&sbar[j % NB], (j / NB) & 1, kWaitLimitNs / 8);
+  }
   if (warp == 1) {
-    // every MMA has completed (already on the normal path; bounded on abort)
-    tc::mbar_wait(drain, 0, abort_flag, kWaitLimitNs / 8);
+    // every MMA has completed (already on the normal path)
+    if (lane == 0) tc::mbar_drain(drain, 0, kWaitLimitNs / 8);
     __syncwarp();
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
-}
-
-// Tile list: expert e contributes ceil(count_e / NT) tiles of up to NT rows.
-__global__ void plan_tiles_kernel(const int32_t* __restrict__ offsets, int E, int NT,
-                                  Tile* __restrict__ tiles, int* __restrict__ n_tiles) {
-  __shared__ int base[257];
-  const int e = threadIdx.x;
-  int cnt = 0;
-  if (e < E) {
-    const int c = offsets[e + 1] - offsets[e];
-    cnt = (c + NT - 1) / NT;
-  }
-  base[e + 1] = cnt;
-  if (e == 0) base[0] = 0;
-  __syncthreads();
-  if (e == 0)
-    for (int i = 1; i <= E; ++i) base[i] += base[i - 1];
-  __syncthreads();
-  if (e < E) {
-    const int r0 = offsets[e], c = offsets[e + 1] - offsets[e];
-    for (int t = 0; t < cnt; ++t) {
-      Tile tl;
-      tl.e = e;
-      tl.row0 = r0 + t * NT;
-      tl.nrows = min(NT, c - t * NT);
-      tl.pad = 0;
-      tiles[base[e] + t] = tl;
-    }
-  }
-  if (e == 0) *n_tiles = base[E];
 }
 
 // Exact two-piece E4M3 split of bf16 rows (see the file comment), written in
@@ -548,11 +704,12 @@ __global__ void plan_tiles_kernel(const int32_t* __restrict__ offsets, int E, in
 // the scale words [2 NT] in the same row order (byte b of a word = E8M0 scale
 // of the window's 32-element block b).  One warp per (padded row, window);
 // lane l holds elements 4l..4l+3 of the window, a block is 8 lanes.  Padded
-// rows get zero pieces.
+// rows get zero pieces.  Row r of the permuted order is src[r], or, with
+// `gather`, src[gather[r] / k] (the layer splits straight from x).
 __global__ void __launch_bounds__(256) split_rows_kernel(
-    const uint16_t* __restrict__ src, int K, const Tile* __restrict__ tiles,
-    const int* __restrict__ n_tiles, int NT, int64_t padded_rows, uint8_t* __restrict__ pieces,
-    uint32_t* __restrict__ words) {
+    const uint16_t* __restrict__ src, const int32_t* __restrict__ gather, int k, int K,
+    const Tile* __restrict__ tiles, const int* __restrict__ n_tiles, int NT, int64_t padded_rows,
+    uint8_t* __restrict__ pieces, uint32_t* __restrict__ words) {
   const int nstg = (K + BKS - 1) / BKS;
   const int st = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -562,11 +719,12 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
   if (ti >= __ldg(n_tiles)) return;
   const Tile tl = tiles[ti];
   const int k0 = stage_k0(st, K);
-  const int k = k0 + lane * 4;
+  const int kk = k0 + lane * 4;
   float v[4] = {0.f, 0.f, 0.f, 0.f};
   if (i < tl.nrows) {
-    const uint2 raw =
-        *reinterpret_cast<const uint2*>(src + static_cast<int64_t>(tl.row0 + i) * K + k);
+    int64_t r = tl.row0 + i;
+    if (gather) r = __ldg(gather + r) / k;
+    const uint2 raw = *reinterpret_cast<const uint2*>(src + r * K + kk);
     v[0] = bf16_to_f32(static_cast<uint16_t>(raw.x));
     v[1] = bf16_to_f32(static_cast<uint16_t>(raw.x >> 16));
     v[2] = bf16_to_f32(static_cast<uint16_t>(raw.y));
@@ -576,26 +734,13 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
   amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
   amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
-  // block exponent floor(log2 amax) - 7 from the biased exponent field; zero
-  // and subnormal blocks take the floor -123, which keeps both scale bytes >= 0
-  const int ebits = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
-  const int t = max(ebits - 127 - 7, -123);
-  const float inv = __uint_as_float(static_cast<uint32_t>(127 - t) << 23);  // 2^-t
-  uint32_t hi4 = 0, lo4 = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float u = v[j] * inv;
-    const __nv_fp8_storage_t h8 = __nv_cvt_float_to_fp8(u, __NV_SATFINITE, __NV_E4M3);
-    const float hf = __half2float(__half(__nv_cvt_fp8_to_halfraw(h8, __NV_E4M3)));
-    const __nv_fp8_storage_t l8 =
-        __nv_cvt_float_to_fp8((u - hf) * 16.0f, __NV_SATFINITE, __NV_E4M3);
-    hi4 |= static_cast<uint32_t>(h8) << (8 * j);
-    lo4 |= static_cast<uint32_t>(l8) << (8 * j);
-  }
+  const int t = split_exponent(amax);
+  uint32_t hi4, lo4;
+  split4(v, t, hi4, lo4);
   // a moved-back last window re-reads [K - 128, 128 st): only its new elements are written
-  if (k >= st * BKS) {
-    *reinterpret_cast<uint32_t*>(pieces + (2 * p) * K + k) = hi4;
-    *reinterpret_cast<uint32_t*>(pieces + (2 * p + 1) * K + k) = lo4;
+  if (kk >= st * BKS) {
+    *reinterpret_cast<uint32_t*>(pieces + (2 * p) * K + kk) = hi4;
+    *reinterpret_cast<uint32_t*>(pieces + (2 * p + 1) * K + kk) = lo4;
   }
   uint32_t whi = 0, wlo = 0;
 #pragma unroll
@@ -613,29 +758,9 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
 
 // ------------------------------------------------------------ host helpers
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      cudaGetLastError();
-      return static_cast<EncodeTiledFn>(nullptr);
-    }
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
 bool encode(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base,
             const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return fn(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box,
@@ -709,155 +834,186 @@ GemmConfig choose_config(const moe_shape& sh) {
       if (smem_bytes(nt, ns, 2, K) <= kMaxSmemPerCta) return {nt, ns, 2};
     for (int ns = kMaxStages; ns >= 2; --ns)
       if (smem_bytes(nt, ns, 1, K) <= kMaxSmemPerCta) return {nt, ns, 1};
-    if (nt == 16) return {16, 0, 1};  // does not fit: rejected at launch
+    if (nt == 16) return {16, 0, 1};  // does not fit: refused by the plan
     nt /= 2;
   }
 }
 
-template <int NT, bool GATE_UP>
-moe_status launch_gemm(const GemmConfig& cfg, const CUtensorMap& mw, const CUtensorMap& mwt,
-                       const CUtensorMap& mx, const uint32_t* words, const uint8_t* scales,
-                       const Tile* tiles, const int* n_tiles, int max_items, int R, int K,
-                       int out_ld, uint16_t* out, int32_t* status, cudaStream_t stream) {
-  const int smem = smem_bytes(NT, cfg.NS, cfg.NB, K);
-  if (cfg.NS < 2 || cfg.NS > kMaxStages || smem > kMaxSmemPerCta) return MOE_ERR_SHAPE;
-  auto kern = grouped_mx_gemm<NT, GATE_UP>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    attr_done = true;
+// The dynamic shared-memory opt-in of a kernel, once per device.
+template <typename Kern>
+bool allow_smem(Kern kern, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
   }
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load() & bit)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemPerCta) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  done.fetch_or(bit);
+  return true;
+}
+
+template <int NT, bool GATE_UP>
+bool prepare_gemm() {
+  static std::atomic<uint64_t> done{0};
+  return allow_smem(grouped_mx_gemm<NT, GATE_UP>, done);
+}
+
+bool prepare_nt(int NT) {
+  switch (NT) {
+    case 16:
+      return prepare_gemm<16, true>() && prepare_gemm<16, false>();
+    case 32:
+      return prepare_gemm<32, true>() && prepare_gemm<32, false>();
+    default:
+      return prepare_gemm<64, true>() && prepare_gemm<64, false>();
+  }
+}
+
+template <int NT, bool GATE_UP>
+moe_status launch_gemm(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& mwt,
+                       const CUtensorMap& mx, const GemmArgs& a, int max_items,
+                       cudaStream_t stream) {
+  const int smem = smem_bytes(NT, P.NS, P.NB, a.K);
   const int grid = max_items < sm_count() ? max_items : sm_count();
   // each CTA holds all 512 tensor-memory columns: ask for enough shared
   // memory that no second CTA shares the SM
   const int smem_launch = smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
-  kern<<<grid, kThreads, smem_launch, stream>>>(mw, mwt, mx, words, scales, tiles, n_tiles, R, K, cfg.NS,
-                                         cfg.NB, out_ld, out, status);
+  grouped_mx_gemm<NT, GATE_UP><<<grid, kThreads, smem_launch, stream>>>(mw, mwt, mx, a);
   return launch_status();
 }
 
 template <bool GATE_UP>
-moe_status launch_nt(const GemmConfig& cfg, const CUtensorMap& mw, const CUtensorMap& mwt,
-                     const CUtensorMap& mx, const uint32_t* words, const uint8_t* scales,
-                     const Tile* tiles, const int* n_tiles, int max_items, int R, int K, int ld,
-                     uint16_t* out, int32_t* status, cudaStream_t st) {
-  switch (cfg.NT) {
+moe_status launch_nt(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& mwt,
+                     const CUtensorMap& mx, const GemmArgs& a, int max_items, cudaStream_t st) {
+  switch (P.NT) {
     case 16:
-      return launch_gemm<16, GATE_UP>(cfg, mw, mwt, mx, words, scales, tiles, n_tiles, max_items,
-                                      R, K, ld, out, status, st);
+      return launch_gemm<16, GATE_UP>(P, mw, mwt, mx, a, max_items, st);
     case 32:
-      return launch_gemm<32, GATE_UP>(cfg, mw, mwt, mx, words, scales, tiles, n_tiles, max_items,
-                                      R, K, ld, out, status, st);
+      return launch_gemm<32, GATE_UP>(P, mw, mwt, mx, a, max_items, st);
     default:
-      return launch_gemm<64, GATE_UP>(cfg, mw, mwt, mx, words, scales, tiles, n_tiles, max_items,
-                                      R, K, ld, out, status, st);
+      return launch_gemm<64, GATE_UP>(P, mw, mwt, mx, a, max_items, st);
   }
 }
 
-struct MlpWs {
-  size_t n_tiles, tiles, pieces, words, total;
+// Workspace of the block-scaled path: the tile list, then for the input rows
+// and for h each its pieces [2 * padded rows][K] and scale words
+// [tiles][K/128 windows][2 NT].
+struct MxWs {
+  size_t n_tiles, tiles, pieces_x, words_x, pieces_h, words_h, total;
   int64_t max_tiles, padded_rows;
 };
 
-MlpWs mlp_ws(const moe_shape& sh) {
+MxWs mx_ws(const moe_shape& sh) {
   const int NT = choose_config(sh).NT;
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
-  const int K = sh.d_model > sh.d_ff ? sh.d_model : sh.d_ff;
-  const int64_t nstg = (K + BKS - 1) / BKS;
-  MlpWs w;
+  const int D = sh.d_model, F = sh.d_ff;
+  MxWs w;
   w.max_tiles = sh.E + (S + NT - 1) / NT;
   w.padded_rows = w.max_tiles * NT;
+  auto words_bytes = [&](int K) {
+    return static_cast<size_t>(w.max_tiles * ((K + BKS - 1) / BKS)) * 2 * NT * 4;
+  };
   w.n_tiles = 0;
   w.tiles = 256;
-  w.pieces = align_up(w.tiles + static_cast<size_t>(w.max_tiles) * sizeof(Tile), 256);
-  w.words = align_up(w.pieces + 2 * static_cast<size_t>(w.padded_rows) * K, 256);
-  w.total = align_up(w.words + static_cast<size_t>(w.max_tiles * nstg) * 2 * NT * 4, 256);
+  w.pieces_x = align_up(w.tiles + static_cast<size_t>(w.max_tiles) * sizeof(Tile), 256);
+  w.words_x = align_up(w.pieces_x + 2 * static_cast<size_t>(w.padded_rows) * D, 256);
+  w.pieces_h = align_up(w.words_x + words_bytes(D), 256);
+  w.words_h = align_up(w.pieces_h + 2 * static_cast<size_t>(w.padded_rows) * F, 256);
+  w.total = align_up(w.words_h + words_bytes(F), 256);
   return w;
-}
-
-moe_status split_launch(const uint16_t* src, int K, const Tile* tiles, const int* n_tiles, int NT,
-                        const MlpWs& W, uint8_t* pieces, uint32_t* words, cudaStream_t stream) {
-  const int nstg = (K + BKS - 1) / BKS;
-  const int64_t blocks = (W.padded_rows + 7) / 8;  // 8 warps per block, one row each
-  split_rows_kernel<<<dim3(static_cast<unsigned>(blocks), nstg), 256, 0, stream>>>(
-      src, K, tiles, n_tiles, NT, W.padded_rows, pieces, words);
-  return launch_status();
-}
-
-moe_status mx_launch(const uint16_t* x_perm, const int32_t* offsets, const moe_shape& sh,
-                     const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
-                     const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
-                     int32_t* status, cudaStream_t stream) {
-  if (sh.T == 0) return MOE_OK;
-  const GemmConfig cfg = choose_config(sh);
-  if (cfg.NS < 2) return MOE_ERR_SHAPE;
-  const int NT = cfg.NT;
-  const MlpWs W = mlp_ws(sh);
-  char* base = static_cast<char*>(ws);
-  int* n_tiles = reinterpret_cast<int*>(base + W.n_tiles);
-  Tile* tiles = reinterpret_cast<Tile*>(base + W.tiles);
-  uint8_t* pieces = reinterpret_cast<uint8_t*>(base + W.pieces);
-  uint32_t* words = reinterpret_cast<uint32_t*>(base + W.words);
-  const int max_tiles = static_cast<int>(W.max_tiles);
-  const int D = sh.d_model, F = sh.d_ff, E = sh.E;
-
-  CUtensorMap m_gu, m_gu_t, m_dn, m_dn_t, m_x, m_h;
-  if (!make_weight_maps(&m_gu, &m_gu_t, wgu_q, E, 2 * F, D, true) ||
-      !make_weight_maps(&m_dn, &m_dn_t, wdn_q, E, D, F, false) ||
-      !make_piece_map(&m_x, pieces, W.padded_rows, D, NT) ||
-      !make_piece_map(&m_h, pieces, W.padded_rows, F, NT))
-    return MOE_ERR_CUDA;
-
-  plan_tiles_kernel<<<1, 256, 0, stream>>>(offsets, E, NT, tiles, n_tiles);
-  moe_status st = launch_status();
-  if (st != MOE_OK) return st;
-  if ((st = split_launch(x_perm, D, tiles, n_tiles, NT, W, pieces, words, stream)) != MOE_OK)
-    return st;
-  const int mt_gu = (F + BN / 2 - 1) / (BN / 2), mt_dn = (D + BN - 1) / BN;
-  st = launch_nt<true>(cfg, m_gu, m_gu_t, m_x, words, wgu_s, tiles, n_tiles, max_tiles * mt_gu,
-                       2 * F, D, F, h, status, stream);
-  if (st != MOE_OK) return st;
-  if ((st = split_launch(h, F, tiles, n_tiles, NT, W, pieces, words, stream)) != MOE_OK) return st;
-  return launch_nt<false>(cfg, m_dn, m_dn_t, m_h, words, wdn_s, tiles, n_tiles, max_tiles * mt_dn,
-                          D, F, D, y_perm, status, stream);
-}
-
-// Shapes with few routed rows per expert (decode) stream the weights once per
-// small token tile and are bound by HBM: they take the block-scaled path
-// above, which moves the codes straight into the tensor core.  Token-heavy
-// shapes (prefill) are bound by the tensor core and take the decode-to-bf16
-// path, whose 2-CTA-per-SM pipeline with 256-token tiles keeps it busier.
-bool native_path(const moe_shape& sh) {
-  const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
-  return 2 * ((S + sh.E - 1) / sh.E) <= 64;
 }
 
 }  // namespace
 
-size_t expert_mlp_bf16_workspace(const moe_shape& sh);
-moe_status expert_mlp_bf16_launch(const uint16_t* x_perm, const int32_t* offsets,
-                                  const moe_shape& sh, const uint8_t* wgu_q, const uint8_t* wgu_s,
-                                  const uint8_t* wdn_q, const uint8_t* wdn_s, uint16_t* h,
-                                  uint16_t* y_perm, void* ws, int32_t* status,
-                                  cudaStream_t stream);
+int mx_tile_width(const moe_shape& sh) { return choose_config(sh).NT; }
+size_t mx_workspace(const moe_shape& sh) { return mx_ws(sh).total; }
 
-size_t expert_mlp_workspace(const moe_shape& sh) {
-  return native_path(sh) ? mlp_ws(sh).total : expert_mlp_bf16_workspace(sh);
+moe_status mx_plan(MlpPlan* p, void* ws) {
+  const moe_shape& sh = p->sh;
+  const GemmConfig cfg = choose_config(sh);
+  if (cfg.NS < 2) return MOE_ERR_SHAPE;
+  const MxWs W = mx_ws(sh);
+  char* base = static_cast<char*>(ws);
+  MxPlan& P = p->mx;
+  P.NT = cfg.NT;
+  P.NS = cfg.NS;
+  P.NB = cfg.NB;
+  P.max_tiles = W.max_tiles;
+  P.padded_rows = W.padded_rows;
+  p->n_tiles = reinterpret_cast<int*>(base + W.n_tiles);
+  p->tiles = reinterpret_cast<Tile*>(base + W.tiles);
+  P.pieces_x = reinterpret_cast<uint8_t*>(base + W.pieces_x);
+  P.words_x = reinterpret_cast<uint32_t*>(base + W.words_x);
+  P.pieces_h = reinterpret_cast<uint8_t*>(base + W.pieces_h);
+  P.words_h = reinterpret_cast<uint32_t*>(base + W.words_h);
+  const int D = sh.d_model, F = sh.d_ff, E = sh.E;
+  if (!make_weight_maps(&P.m_gu, &P.m_gu_t, p->wgu_q, E, 2 * F, D, true) ||
+      !make_weight_maps(&P.m_dn, &P.m_dn_t, p->wdn_q, E, D, F, false) ||
+      !make_piece_map(&P.m_x, P.pieces_x, W.padded_rows, D, cfg.NT) ||
+      !make_piece_map(&P.m_h, P.pieces_h, W.padded_rows, F, cfg.NT))
+    return MOE_ERR_CUDA;
+  if (!prepare_nt(cfg.NT)) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
-moe_status expert_mlp_launch(const uint16_t* x_perm, const int32_t* offsets, const moe_shape& sh,
-                             const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
-                             const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
-                             int32_t* status, cudaStream_t stream) {
-  if (native_path(sh))
-    return mx_launch(x_perm, offsets, sh, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm, ws, status,
-                     stream);
-  return expert_mlp_bf16_launch(x_perm, offsets, sh, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm, ws,
-                                status, stream);
+moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int fail_cta,
+                      cudaStream_t stream) {
+  const MxPlan& P = p.mx;
+  const moe_shape& sh = p.sh;
+  const int NT = P.NT, D = sh.d_model, F = sh.d_ff, E = sh.E;
+  moe_status st;
+  if (!in.tiles_ready &&
+      (st = plan_tiles_launch(in.offsets, E, NT, p.tiles, p.n_tiles, stream)) != MOE_OK)
+    return st;
+  // the input rows, split into pieces (straight from x inside the layer)
+  {
+    const bool from_x = in.x != nullptr;
+    const int nwin = (D + BKS - 1) / BKS;
+    const int64_t blocks = (P.padded_rows + 7) / 8;  // 8 warps per block, one row each
+    split_rows_kernel<<<dim3(static_cast<unsigned>(blocks), nwin), 256, 0, stream>>>(
+        from_x ? in.x : p.x_perm, from_x ? in.sorted_slot : nullptr, from_x ? in.k : 1, D,
+        p.tiles, p.n_tiles, NT, P.padded_rows, P.pieces_x, P.words_x);
+    if ((st = launch_status()) != MOE_OK) return st;
+  }
+  const int max_tiles = static_cast<int>(P.max_tiles);
+  const int mt_gu = (F + BN / 2 - 1) / (BN / 2), mt_dn = (D + BN - 1) / BN;
+  GemmArgs a{};
+  a.tiles = p.tiles;
+  a.n_tiles = p.n_tiles;
+  a.NS = P.NS;
+  a.NB = P.NB;
+  a.status = status;
+  // gate/up + SwiGLU: h (when asked) and the pieces of h
+  a.sfx_words = P.words_x;
+  a.scales = p.wgu_s;
+  a.wq = p.wgu_q;
+  a.rows_per_expert = 2 * F;
+  a.K = D;
+  a.out_ld = F;
+  a.out = p.h;
+  a.pieces_out = P.pieces_h;
+  a.words_out = P.words_h;
+  a.fail_cta = fail_cta;
+  if ((st = launch_nt<true>(P, P.m_gu, P.m_gu_t, P.m_x, a, max_tiles * mt_gu, stream)) != MOE_OK)
+    return st;
+  // down
+  a.sfx_words = P.words_h;
+  a.scales = p.wdn_s;
+  a.wq = p.wdn_q;
+  a.rows_per_expert = D;
+  a.K = F;
+  a.out_ld = D;
+  a.out = p.y_perm;
+  a.pieces_out = nullptr;
+  a.words_out = nullptr;
+  a.fail_cta = -1;
+  return launch_nt<false>(P, P.m_dn, P.m_dn_t, P.m_h, a, max_tiles * mt_dn, stream);
 }
 
 }  // namespace moe

@@ -43,7 +43,10 @@
 // MOE_ERR_TIMEOUT in the status word, drains its copies and returns.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
+#include "mlp_plan.cuh"
 #include "tc_sm100.cuh"
 
 namespace moe {
@@ -57,10 +60,7 @@ constexpr int kDecodeGroups = 3;
 constexpr int kDecWarp0 = 4;
 constexpr int kThreads = 32 * (kDecWarp0 + 4 * kDecodeGroups);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
-struct Tile {
-  int e, row0, nrows, pad;
-};
+constexpr uint64_t kTestWaitNs = 200000ull;  // the injected wait of test_timeout_cta
 
 // per token-tile width: token/A slots and MMA issuers (tensor memory holds
 // NMMA accumulators of NT columns plus NA A slots of 32 columns)
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
                        const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ scales,
                        const Tile* __restrict__ tiles, const int* __restrict__ n_tiles,
                        int rows_per_expert, int K, int out_ld, uint16_t* __restrict__ out,
-                       int32_t* __restrict__ status) {
+                       int32_t* __restrict__ status, int fail_cta) {
   constexpr int NA = slots_for(NT);
   constexpr int NMMA = issuers_for(NT);
   constexpr int X_STAGE = NT * 128;
@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
   uint64_t* consumed = afull + NA;     // [NA]  MMA done with token slot + A slot
   uint64_t* sbar = consumed + NA;      // scales landed
   uint64_t* dfull = sbar + 1;          // accumulators complete (one commit per issuer)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(dfull + 1);
+  uint64_t* never = dfull + 1;         // completed by nothing (the injected test wait)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
     }
     tc::mbar_init(sbar, 1);
     tc::mbar_init(dfull, NMMA);
+    tc::mbar_init(never, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
     tc::tma_prefetch_desc(&map_w);
@@ -249,8 +251,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
       }
       // drain: every copy this thread issued has landed before the CTA exits
       for (int kb = max(0, issued - NSW); kb < issued; ++kb)
-        tc::mbar_wait(&wfull[kb % NSW], (kb / NSW) & 1, abort_flag, kWaitLimitNs / 8);
-      tc::mbar_wait(sbar, 0, abort_flag, kWaitLimitNs / 8);
+        tc::mbar_drain(&wfull[kb % NSW], (kb / NSW) & 1, kWaitLimitNs / 8);
+      tc::mbar_drain(sbar, 0, kWaitLimitNs / 8);
     }
   } else if (warp == 1) {
     // --------------------------------------------------- token producer
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
         ++issued;
       }
       for (int kb = max(0, issued - NA); kb < issued; ++kb)
-        tc::mbar_wait(&xfull[kb % NA], (kb / NA) & 1, abort_flag, kWaitLimitNs / 8);
+        tc::mbar_drain(&xfull[kb % NA], (kb / NA) & 1, kWaitLimitNs / 8);
     }
   } else if (warp < kDecWarp0) {
     // ---------------------------------------------------------- MMA issuers
@@ -275,7 +277,16 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
     if (lane == 0 && mi < NMMA) {
       const uint32_t tmem_d = tmem + mi * NT;
       int done = 0;
-      for (int kb = mi; kb < KB; kb += NMMA) {
+      bool ok = true;
+      // testing only: the first wait of this CTA's first issuer waits on a
+      // barrier that nothing completes, with a short limit, and gives up as a
+      // timeout would
+      if (mi == 0 && static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x) == fail_cta &&
+          !tc::mbar_wait(never, 0, abort_flag, kTestWaitNs)) {
+        abort_cta(abort_flag, status);
+        ok = false;
+      }
+      for (int kb = mi; ok && kb < KB; kb += NMMA) {
         const int j = kb % NA;
         const uint32_t par = (kb / NA) & 1;
         if (!tc::mbar_wait(&xfull[j], par, abort_flag, kWaitLimitNs) ||
@@ -435,69 +446,20 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
   __syncthreads();
   if (warp == 1) {
     // the accumulator barrier completes once every issued MMA has finished
-    // (already observed on the normal path; bounded on the abort path)
-    tc::mbar_wait(dfull, 0, abort_flag, kWaitLimitNs / 8);
+    // (already observed on the normal path)
+    tc::mbar_drain(dfull, 0, kWaitLimitNs / 8);
     __syncwarp();
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
-// Tile list: expert e contributes ceil(count_e / NT) tiles of up to NT rows.
-__global__ void plan_tiles_kernel(const int32_t* __restrict__ offsets, int E, int NT,
-                                  Tile* __restrict__ tiles, int* __restrict__ n_tiles) {
-  __shared__ int base[257];
-  const int e = threadIdx.x;
-  int cnt = 0;
-  if (e < E) {
-    const int c = offsets[e + 1] - offsets[e];
-    cnt = (c + NT - 1) / NT;
-  }
-  base[e + 1] = cnt;
-  if (e == 0) base[0] = 0;
-  __syncthreads();
-  if (e == 0)
-    for (int i = 1; i <= E; ++i) base[i] += base[i - 1];
-  __syncthreads();
-  if (e < E) {
-    const int r0 = offsets[e], c = offsets[e + 1] - offsets[e];
-    for (int t = 0; t < cnt; ++t) {
-      Tile tl;
-      tl.e = e;
-      tl.row0 = r0 + t * NT;
-      tl.nrows = min(NT, c - t * NT);
-      tl.pad = 0;
-      tiles[base[e] + t] = tl;
-    }
-  }
-  if (e == 0) *n_tiles = base[E];
-}
 
 // ------------------------------------------------------------ host helpers
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      cudaGetLastError();
-      return static_cast<EncodeTiledFn>(nullptr);
-    }
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
 // packed codes [E][R][K/2] bytes, box = (BK/2 bytes, box_rows rows, 1 expert)
 bool make_weight_map(CUtensorMap* map, const uint8_t* q, int E, int R, int K, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(R),
                               static_cast<cuuint64_t>(E)};
@@ -512,7 +474,7 @@ bool make_weight_map(CUtensorMap* map, const uint8_t* q, int E, int R, int K, in
 
 // token rows [rows][K] bf16, box = (BK elements, NT rows), 128-byte swizzle
 bool make_token_map(CUtensorMap* map, const uint16_t* x, int64_t rows, int K, int NT) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
@@ -535,97 +497,132 @@ int choose_nt(const moe_shape& sh) {
   return nt;
 }
 
+// The dynamic shared-memory opt-in of both kernels of a tile width, once per
+// device.
+template <int NT>
+bool prepare_gemm() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load() & bit)) return true;
+  if (cudaFuncSetAttribute(grouped_mxfp4_gemm<NT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           227 * 1024) != cudaSuccess ||
+      cudaFuncSetAttribute(grouped_mxfp4_gemm<NT, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  done.fetch_or(bit);
+  return true;
+}
+
+bool prepare_nt(int NT) {
+  switch (NT) {
+    case 32:
+      return prepare_gemm<32>();
+    case 64:
+      return prepare_gemm<64>();
+    case 128:
+      return prepare_gemm<128>();
+    default:
+      return prepare_gemm<256>();
+  }
+}
+
 template <int NT, bool GATE_UP>
 moe_status launch_gemm(const CUtensorMap& mw, const CUtensorMap& mx, const uint8_t* scales,
                        const Tile* tiles, const int* n_tiles, int grid_x, int grid_y, int R, int K,
-                       int out_ld, uint16_t* out, int32_t* status, cudaStream_t stream) {
+                       int out_ld, uint16_t* out, int32_t* status, int fail_cta,
+                       cudaStream_t stream) {
   const int smem = smem_layout(NT, K).total + 1024;
-  if (smem > 227 * 1024) return MOE_ERR_SHAPE;
-  auto kern = grouped_mxfp4_gemm<NT, GATE_UP>;
-  static bool attr_done = false;
-  static int attr_smem = 0;
-  if (!attr_done || attr_smem < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    attr_done = true;
-    attr_smem = 227 * 1024;
-  }
-  kern<<<dim3(grid_x, grid_y), kThreads, smem, stream>>>(mw, mx, scales, tiles, n_tiles, R, K,
-                                                          out_ld, out, status);
+  grouped_mxfp4_gemm<NT, GATE_UP><<<dim3(grid_x, grid_y), kThreads, smem, stream>>>(
+      mw, mx, scales, tiles, n_tiles, R, K, out_ld, out, status, fail_cta);
   return launch_status();
 }
 
 template <bool GATE_UP>
 moe_status launch_nt(int NT, const CUtensorMap& mw, const CUtensorMap& mx, const uint8_t* scales,
                      const Tile* tiles, const int* n_tiles, int gx, int gy, int R, int K, int ld,
-                     uint16_t* out, int32_t* status, cudaStream_t st) {
+                     uint16_t* out, int32_t* status, int fail_cta, cudaStream_t st) {
   switch (NT) {
     case 32:
       return launch_gemm<32, GATE_UP>(mw, mx, scales, tiles, n_tiles, gx, gy, R, K, ld, out,
-                                      status, st);
+                                      status, fail_cta, st);
     case 64:
       return launch_gemm<64, GATE_UP>(mw, mx, scales, tiles, n_tiles, gx, gy, R, K, ld, out,
-                                      status, st);
+                                      status, fail_cta, st);
     case 128:
       return launch_gemm<128, GATE_UP>(mw, mx, scales, tiles, n_tiles, gx, gy, R, K, ld, out,
-                                       status, st);
+                                       status, fail_cta, st);
     default:
       return launch_gemm<256, GATE_UP>(mw, mx, scales, tiles, n_tiles, gx, gy, R, K, ld, out,
-                                       status, st);
+                                       status, fail_cta, st);
   }
 }
 
-struct MlpWs {
-  size_t status, n_tiles, tiles, total;
+// Workspace of this path: the tile count and the tile list.
+struct BfWs {
+  size_t n_tiles, tiles, total;
+  int64_t max_tiles;
 };
 
-MlpWs mlp_ws(const moe_shape& sh) {
+BfWs bf_ws(const moe_shape& sh) {
   const int NT = choose_nt(sh);
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
-  const int64_t max_tiles = sh.E + (S + NT - 1) / NT;
-  MlpWs w;
-  w.status = 0;
-  w.n_tiles = 16;
+  BfWs w;
+  w.max_tiles = sh.E + (S + NT - 1) / NT;
+  w.n_tiles = 0;
   w.tiles = 256;
-  w.total = align_up(w.tiles + static_cast<size_t>(max_tiles) * sizeof(Tile), 256);
+  w.total = align_up(w.tiles + static_cast<size_t>(w.max_tiles) * sizeof(Tile), 256);
   return w;
 }
 
 }  // namespace
 
-size_t expert_mlp_bf16_workspace(const moe_shape& sh) { return mlp_ws(sh).total; }
+int bf_tile_width(const moe_shape& sh) { return choose_nt(sh); }
+size_t bf_workspace(const moe_shape& sh) { return bf_ws(sh).total; }
 
-moe_status expert_mlp_bf16_launch(const uint16_t* x_perm, const int32_t* offsets, const moe_shape& sh,
-                             const uint8_t* wgu_q, const uint8_t* wgu_s, const uint8_t* wdn_q,
-                             const uint8_t* wdn_s, uint16_t* h, uint16_t* y_perm, void* ws,
-                             int32_t* status, cudaStream_t stream) {
-  if (sh.T == 0) return MOE_OK;
+moe_status bf_plan(MlpPlan* p, void* ws) {
+  const moe_shape& sh = p->sh;
   const int NT = choose_nt(sh);
-  const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
-  const MlpWs W = mlp_ws(sh);
+  const int K = sh.d_model > sh.d_ff ? sh.d_model : sh.d_ff;
+  if (smem_layout(NT, K).total + 1024 > 227 * 1024) return MOE_ERR_SHAPE;
+  const BfWs W = bf_ws(sh);
   char* base = static_cast<char*>(ws);
-  int* n_tiles = reinterpret_cast<int*>(base + W.n_tiles);
-  Tile* tiles = reinterpret_cast<Tile*>(base + W.tiles);
-  const int max_tiles = static_cast<int>(sh.E + (S + NT - 1) / NT);
+  BfPlan& P = p->bf;
+  P.NT = NT;
+  P.max_tiles = W.max_tiles;
+  p->n_tiles = reinterpret_cast<int*>(base + W.n_tiles);
+  p->tiles = reinterpret_cast<Tile*>(base + W.tiles);
+  const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
   const int D = sh.d_model, F = sh.d_ff, E = sh.E;
-
-  CUtensorMap m_gu, m_x, m_dn, m_h;
-  if (!make_weight_map(&m_gu, wgu_q, E, 2 * F, D, 64) ||
-      !make_token_map(&m_x, x_perm, S, D, NT) || !make_weight_map(&m_dn, wdn_q, E, D, F, BM) ||
-      !make_token_map(&m_h, h, S, F, NT))
+  if (!make_weight_map(&P.m_gu, p->wgu_q, E, 2 * F, D, 64) ||
+      !make_token_map(&P.m_x, p->x_perm, S, D, NT) ||
+      !make_weight_map(&P.m_dn, p->wdn_q, E, D, F, BM) || !make_token_map(&P.m_h, p->h, S, F, NT))
     return MOE_ERR_CUDA;
+  if (!prepare_nt(NT)) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
 
-  plan_tiles_kernel<<<1, 256, 0, stream>>>(offsets, E, NT, tiles, n_tiles);
-  moe_status st = launch_status();
+moe_status bf_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int fail_cta,
+                      cudaStream_t stream) {
+  const BfPlan& P = p.bf;
+  const moe_shape& sh = p.sh;
+  const int NT = P.NT, D = sh.d_model, F = sh.d_ff, E = sh.E;
+  const int max_tiles = static_cast<int>(P.max_tiles);
+  moe_status st;
+  if (!in.tiles_ready &&
+      (st = plan_tiles_launch(in.offsets, E, NT, p.tiles, p.n_tiles, stream)) != MOE_OK)
+    return st;
+  st = launch_nt<true>(NT, P.m_gu, P.m_x, p.wgu_s, p.tiles, p.n_tiles, F / 64, max_tiles, 2 * F,
+                       D, F, p.h, status, fail_cta, stream);
   if (st != MOE_OK) return st;
-  st = launch_nt<true>(NT, m_gu, m_x, wgu_s, tiles, n_tiles, F / 64, max_tiles, 2 * F, D, F, h,
-                       status, stream);
-  if (st != MOE_OK) return st;
-  return launch_nt<false>(NT, m_dn, m_h, wdn_s, tiles, n_tiles, (D + BM - 1) / BM, max_tiles, D,
-                          F, D, y_perm, status, stream);
+  return launch_nt<false>(NT, P.m_dn, P.m_h, p.wdn_s, p.tiles, p.n_tiles, (D + BM - 1) / BM,
+                          max_tiles, D, F, D, p.y_perm, status, -1, stream);
 }
 
 }  // namespace moe

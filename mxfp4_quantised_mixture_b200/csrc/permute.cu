@@ -15,8 +15,12 @@
 //      expert find each other with __match_any_sync, rank themselves by lane
 //      order, and the group leader advances the run.  Chunks are contiguous
 //      and walked in order, so positions follow ascending slot index.
+// Inside the layer the same CTA also writes the grouped GEMMs' tile list
+// (expert e gets ceil(count_e / NT) tiles of up to NT rows), which saves the
+// GEMMs a launch of their own.
 // The row gather (HBM-bound) runs as a separate full-GPU kernel.
 #include "common.cuh"
+#include "mlp_plan.cuh"
 
 namespace moe {
 namespace {
@@ -28,9 +32,11 @@ constexpr int kMaxE = 256;
 __global__ void __launch_bounds__(kThreads, 1)
     permute_kernel(const int32_t* __restrict__ idx, int64_t S, int E, int32_t* __restrict__ counts,
                    int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_slot,
-                   int32_t* __restrict__ slot_pos) {
+                   int32_t* __restrict__ slot_pos, int NT, Tile* __restrict__ tiles,
+                   int* __restrict__ n_tiles) {
   __shared__ int32_t cnt[kWarps][kMaxE];  // per (warp, expert) count, then running position
   __shared__ int32_t off[kMaxE + 1];
+  __shared__ int32_t tbase[kMaxE + 1];    // first tile of each expert (tile list only)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&cnt[0][0])[i] = 0;
   __syncthreads();
@@ -66,6 +72,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   for (int e = threadIdx.x; e <= E; e += kThreads) offsets[e] = off[e];
+  if (tiles) {
+    // tile list: per-expert tile counts, their exclusive scan (warp 0), then
+    // expert e's tiles written by thread e
+    if (warp == 0) {
+      int carry = 0;
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int nt = e < E ? (off[e + 1] - off[e] + NT - 1) / NT : 0;
+        int incl = nt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        if (e < E) tbase[e] = carry + incl - nt;
+        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      if (lane == 0) *n_tiles = carry;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+      const int r0 = off[e], c = off[e + 1] - off[e];
+      for (int t = 0; t * NT < c; ++t) {
+        Tile tl;
+        tl.e = e;
+        tl.row0 = r0 + t * NT;
+        tl.nrows = min(NT, c - t * NT);
+        tl.pad = 0;
+        tiles[tbase[e] + t] = tl;
+      }
+    }
+  }
   // column scan: first position of each (warp, expert) run
   for (int e = threadIdx.x; e < E; e += kThreads) {
     int run = off[e];
@@ -119,11 +157,13 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 
 moe_status permute_launch(const int32_t* idx, const uint16_t* x, const moe_shape& sh,
                           int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
-                          int32_t* slot_pos, uint16_t* x_perm, cudaStream_t stream) {
+                          int32_t* slot_pos, uint16_t* x_perm, int NT, Tile* tiles,
+                          int* n_tiles, cudaStream_t stream) {
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
-  permute_kernel<<<1, kThreads, 0, stream>>>(idx, S, sh.E, counts, offsets, sorted_slot, slot_pos);
+  permute_kernel<<<1, kThreads, 0, stream>>>(idx, S, sh.E, counts, offsets, sorted_slot, slot_pos,
+                                             NT, tiles, n_tiles);
   moe_status st = launch_status();
-  if (st != MOE_OK || S == 0) return st;
+  if (st != MOE_OK || S == 0 || x_perm == nullptr) return st;
   const int vec = sh.d_model / 8;
   int64_t want = (S * 32 + 255) / 256;
   int64_t cap = static_cast<int64_t>(sm_count()) * 8;
@@ -152,6 +192,6 @@ extern "C" moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x, mo
   if (need > 0 && (ws == nullptr || ws_bytes < need)) return MOE_ERR_WORKSPACE;
   moe_status st = check_device();
   if (st != MOE_OK) return st;
-  return permute_launch(topk_idx, x, shape, counts, offsets, sorted_slot, slot_pos, x_perm,
-                        static_cast<cudaStream_t>(stream));
+  return permute_launch(topk_idx, x, shape, counts, offsets, sorted_slot, slot_pos, x_perm, 0,
+                        nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }

@@ -24,7 +24,11 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
 
 __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ logits, int T,
                                                         int E, int k, int32_t* __restrict__ idx,
-                                                        float* __restrict__ w) {
+                                                        float* __restrict__ w,
+                                                        int32_t* __restrict__ clear_status) {
+  // inside the layer the routing is the first kernel: it resets the layer's
+  // device status word, which the later kernels only ever set to an error
+  if (clear_status && blockIdx.x == 0 && threadIdx.x == 0) *clear_status = MOE_OK;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -58,7 +62,9 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
         bi = oi;
       }
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    // bi stays out of range only if this lane's remaining logits are NaN
+    // (a violated precondition): nothing is marked taken then
+    if (bi < E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
     if (j == 0) top = bv;
     if (lane == j) {
       my_idx = bi;
@@ -78,10 +84,10 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
 }  // namespace
 
 moe_status route_launch(const float* logits, int T, int E, int k, int32_t* idx, float* w,
-                        cudaStream_t stream) {
+                        int32_t* clear_status, cudaStream_t stream) {
   if (T == 0) return MOE_OK;
   const int grid = (T + kThreads / 32 - 1) / (kThreads / 32);
-  route_kernel<<<grid, kThreads, 0, stream>>>(logits, T, E, k, idx, w);
+  route_kernel<<<grid, kThreads, 0, stream>>>(logits, T, E, k, idx, w, clear_status);
   return launch_status();
 }
 
@@ -102,5 +108,6 @@ extern "C" moe_status moe_route(const float* logits, int32_t T, int32_t E, int32
   if (!aligned16(logits) || !aligned16(topk_idx) || !aligned16(topk_w)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_device();
   if (st != MOE_OK) return st;
-  return route_launch(logits, T, E, k, topk_idx, topk_w, static_cast<cudaStream_t>(stream));
+  return route_launch(logits, T, E, k, topk_idx, topk_w, nullptr,
+                      static_cast<cudaStream_t>(stream));
 }

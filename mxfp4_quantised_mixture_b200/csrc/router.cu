@@ -7,12 +7,17 @@
 // The router scores every token against every expert; the routing that
 // follows is the one moe_route computes from given logits.
 //
-// One CTA per 128 tokens.  The scores are a bf16 GEMM on the tensor core:
+// One cluster of up to 8 CTAs per 128 tokens, each CTA taking a contiguous
+// share of the reduction axis (so a decode batch of a few tokens still
+// spreads over several SMs).  The scores are a bf16 GEMM on the tensor core:
 // tokens on the MMA's M side (128), the experts on N (E padded to a multiple
 // of 16, at most 256), K = D in stages of 64 (one 128-byte swizzle row of
 // bf16), both operands by TMA into shared memory, the fp32 accumulator in
-// tensor memory.  Four epilogue warps give each token row to one thread,
-// which reads its E scores from tensor memory, keeps a running top-8 list in
+// tensor memory.  Each CTA moves its partial scores from tensor memory to its
+// shared memory; after a cluster barrier the CTA that owns a token (rank
+// token % cluster size) adds the partials over distributed shared memory in
+// rank order, a fixed order, so the scores do not depend on scheduling.
+// One thread per token row keeps a running top-8 list in
 // registers (value descending, index ascending), and applies the softmax
 // over the first k in fp32 with the same summation order as moe_route, so
 // the routing equals moe_route applied to the returned logits.
@@ -20,6 +25,8 @@
 // in the status word and returns after draining its copies and MMAs.
 #include <cuda.h>
 #include <math.h>
+
+#include <atomic>
 
 #include "common.cuh"
 #include "tc_sm100.cuh"
@@ -58,8 +65,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* dfull = empty + NSR;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(dfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // the partial scores of this CTA, [npad][MT] fp32, over the ring once every
+  // stage is consumed (the ring holds 64 KB + 512 npad bytes, the partials
+  // 512 npad)
+  float* part = reinterpret_cast<float*>(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nstg = D / BKR;
+  // this CTA's share of K: stages [st0, st1) of the cluster's cs CTAs
+  const int cs = gridDim.y, rank = blockIdx.y;
+  const int nstg_all = D / BKR;
+  const int st0 = rank * nstg_all / cs, st1 = (rank + 1) * nstg_all / cs;
+  const int nstg = st1 - st0;
   const int t0 = blockIdx.x * MT;
   int tcols = 32;
   while (tcols < npad) tcols *= 2;
@@ -87,28 +102,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       int issued = 0;
-      for (int st = 0; st < nstg; ++st) {
-        const int s = st % NSR, u = st / NSR;
+      for (int j = 0; j < nstg; ++j) {
+        const int s = j % NSR, u = j / NSR;
         if (u > 0 && !tc::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitLimitNs)) {
           *abort_flag = 1;
           record_status(status, MOE_ERR_TIMEOUT);
           break;
         }
         tc::mbar_arrive_expect_tx(&full[s], A_BYTES + b_bytes);
-        tc::tma_load_2d(as + s * A_BYTES, &map_x, &full[s], st * BKR, t0);
-        tc::tma_load_2d(bs + s * b_bytes, &map_w, &full[s], st * BKR, 0);
+        tc::tma_load_2d(as + s * A_BYTES, &map_x, &full[s], (st0 + j) * BKR, t0);
+        tc::tma_load_2d(bs + s * b_bytes, &map_w, &full[s], (st0 + j) * BKR, 0);
         ++issued;
       }
-      for (int st = max(0, issued - NSR); st < issued; ++st)
-        tc::mbar_wait(&full[st % NSR], (st / NSR) & 1, abort_flag, kWaitLimitNs / 8);
+      for (int j = max(0, issued - NSR); j < issued; ++j)
+        tc::mbar_drain(&full[j % NSR], (j / NSR) & 1, kWaitLimitNs / 8);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(MT, npad);
       int done = 0;
-      for (int st = 0; st < nstg; ++st) {
-        const int s = st % NSR;
-        if (!tc::mbar_wait(&full[s], (st / NSR) & 1, abort_flag, kWaitLimitNs)) {
+      for (int j = 0; j < nstg; ++j) {
+        const int s = j % NSR;
+        if (!tc::mbar_wait(&full[s], (j / NSR) & 1, abort_flag, kWaitLimitNs)) {
           *abort_flag = 1;
           record_status(status, MOE_ERR_TIMEOUT);
           break;
@@ -119,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // a descriptor addresses shared memory in 16-byte units: +2 per 16 bf16
 #pragma unroll
         for (int kk = 0; kk < BKR / 16; ++kk)
-          tc::mma_bf16_ss(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (st | kk) != 0);
+          tc::mma_bf16_ss(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (j | kk) != 0);
         tc::mma_commit(&empty[s]);
         ++done;
       }
@@ -129,14 +144,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive(dfull);
     }
   } else {
+    // this CTA's partial scores: accumulator row m (token t0 + m) -> part[e][m]
     const int q = warp & 3;
     const int m = q * 32 + lane;
-    const int t = t0 + m;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     bool ok = tc::mbar_wait(dfull, 0, abort_flag, kWaitLimitNs);
     ok = __all_sync(0xFFFFFFFFu, ok) && *abort_flag == 0;
     if (ok) {
       tc::tc_fence_after();
+      for (int c = 0; c < npad; c += 16) {
+        uint32_t r[16];
+        tc::tmem_ld16(tmem + lane_base + c, r);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) part[(c + i) * MT + m] = __uint_as_float(r[i]);
+      }
+    }
+  }
+
+  // every CTA's partials are in its shared memory
+  tc::tc_fence_before();
+  tc::cluster_sync();
+
+  if (warp >= 2) {
+    // token m belongs to the CTA of rank m % cs: it adds the cs partial
+    // scores in rank order (fixed, so the scores do not depend on scheduling),
+    // keeps a running top-8 list and applies the softmax over the first k
+    const int q = warp & 3;
+    const int m = q * 32 + lane;
+    const int t = t0 + m;
+    if (m % cs == rank && t < T && *abort_flag == 0) {
       float tv[8];
       int ti[8];
 #pragma unroll
@@ -144,57 +181,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         tv[j] = -INFINITY;
         ti[j] = 0x7FFFFFFF;
       }
-      for (int c = 0; c < npad; c += 16) {
-        uint32_t r[16];
-        tc::tmem_ld16(tmem + lane_base + c, r);
-        tc::tmem_ld_wait();
+      for (int e = 0; e < E; ++e) {
+        const float* pe = part + e * MT + m;
+        float v = tc::ld_cluster_f32(tc::cluster_addr(pe, 0));
+        for (int r = 1; r < cs; ++r) v += tc::ld_cluster_f32(tc::cluster_addr(pe, r));
+        if (logits) logits[static_cast<int64_t>(t) * E + e] = v;
+        // experts arrive in index order: an equal value never displaces an
+        // earlier one, so ties keep the lower index
+        if (better(v, e, tv[7], ti[7])) {
+          tv[7] = v;
+          ti[7] = e;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int e = c + i;
-          if (e >= E) break;
-          const float v = __uint_as_float(r[i]);
-          if (logits && t < T) logits[static_cast<int64_t>(t) * E + e] = v;
-          // experts arrive in index order: an equal value never displaces an
-          // earlier one, so ties keep the lower index
-          if (better(v, e, tv[7], ti[7])) {
-            tv[7] = v;
-            ti[7] = e;
-#pragma unroll
-            for (int j = 7; j > 0; --j) {
-              if (better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
-                const float fv = tv[j];
-                tv[j] = tv[j - 1];
-                tv[j - 1] = fv;
-                const int fi = ti[j];
-                ti[j] = ti[j - 1];
-                ti[j - 1] = fi;
-              }
+          for (int j = 7; j > 0; --j) {
+            if (better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
+              const float fv = tv[j];
+              tv[j] = tv[j - 1];
+              tv[j - 1] = fv;
+              const int fi = ti[j];
+              ti[j] = ti[j - 1];
+              ti[j - 1] = fi;
             }
           }
         }
       }
-      if (t < T) {
-        // softmax over the first k, summed in the order of moe_route's
-        // butterfly over lanes j = 0..7 (zero beyond k)
-        float ex[8];
+      // softmax over the first k, summed in the order of moe_route's
+      // butterfly over lanes j = 0..7 (zero beyond k)
+      float ex[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ex[j] = j < k ? expf(tv[j] - tv[0]) : 0.f;
-        const float z = ((ex[0] + ex[4]) + (ex[2] + ex[6])) + ((ex[1] + ex[5]) + (ex[3] + ex[7]));
+      for (int j = 0; j < 8; ++j) ex[j] = j < k ? expf(tv[j] - tv[0]) : 0.f;
+      const float z = ((ex[0] + ex[4]) + (ex[2] + ex[6])) + ((ex[1] + ex[5]) + (ex[3] + ex[7]));
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < k) {
-            idx[static_cast<int64_t>(t) * k + j] = ti[j];
-            wts[static_cast<int64_t>(t) * k + j] = ex[j] / z;
-          }
+      for (int j = 0; j < 8; ++j) {
+        if (j < k) {
+          idx[static_cast<int64_t>(t) * k + j] = ti[j];
+          wts[static_cast<int64_t>(t) * k + j] = ex[j] / z;
         }
       }
     }
   }
 
-  tc::tc_fence_before();
-  __syncthreads();
+  // no CTA leaves while another may still read its partials
+  tc::cluster_sync();
   if (warp == 1) {
-    tc::mbar_wait(dfull, 0, abort_flag, kWaitLimitNs / 8);
+    if (lane == 0) tc::mbar_drain(dfull, 0, kWaitLimitNs / 8);
     __syncwarp();
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, tcols);
@@ -244,18 +273,45 @@ moe_status router_launch(const uint16_t* x, const uint16_t* w_router, int T, int
   CUtensorMap mx, mw;
   if (!make_rows_map(&mx, x, T, D, MT) || !make_rows_map(&mw, w_router, E, D, npad))
     return MOE_ERR_CUDA;
-  static bool attr_done = false;
-  if (!attr_done) {
+  // the dynamic shared-memory opt-in, once per device
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (!bit || !(attr_done.load() & bit)) {
     if (cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_bytes_router(256)) != cudaSuccess) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
-    attr_done = true;
+    attr_done.fetch_or(bit);
   }
-  const int grid = (T + MT - 1) / MT;
-  router_kernel<<<grid, kThreads, smem_bytes_router(npad), stream>>>(mx, mw, T, D, E, npad, k,
-                                                                     logits, idx, wts, status);
+  // one cluster of cs CTAs per 128 tokens splits K: about one SM per CTA
+  // overall, at most 8 per cluster, at least one 64-K stage each
+  const int nblk = (T + MT - 1) / MT;
+  int cs = (sm_count() + nblk - 1) / nblk;
+  cs = cs < 1 ? 1 : (cs > 8 ? 8 : cs);
+  if (cs > D / BKR) cs = D / BKR;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nblk, cs, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes_router(npad);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = cs;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, router_kernel, mx, mw, T, D, E, npad, k, logits, idx, wts,
+                         status) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
   return launch_status();
 }
 

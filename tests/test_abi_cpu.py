@@ -24,7 +24,7 @@ def declared_functions():
 def test_header_declares_the_six_calls_and_helpers():
     names = declared_functions()
     for n in ["mxfp4_quantize", "mxfp4_quantize_sr_rht", "moe_route", "moe_permute",
-              "moe_expert_mlp", "moe_combine",
+              "moe_expert_mlp", "moe_expert_mlp_ex", "moe_combine", "moe_layer_static_status",
               "moe_layer_forward", "moe_workspace_size", "moe_status_string"]:
         assert n in names
 
@@ -105,6 +105,31 @@ def test_bad_arguments_rejected_before_the_device():
     assert L.moe_expert_mlp(16, 16, sh, 32, 16, 32, 16, 16, 16, 16, mlp - 1, None) == moe.MOE_ERR_WORKSPACE
     assert L.moe_combine(16, 16, 16, sh, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_permute(16, 16, sh, None, 16, 16, 16, 16, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_static_status(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_static_status(18, None) == moe.MOE_ERR_INVALID_ARG  # not 4-byte aligned
+
+
+def test_expert_mlp_ex_path_and_workspace_checked_before_the_device():
+    L = moe.lib
+    sh = moe.make_shape(64, 32, 4, 2880, 2880)  # decode-sized: auto = block-scaled
+    bs = moe.moe_workspace_size(sh, moe.WS_EXPERT_MLP_BLOCK_SCALED)
+    bf = moe.moe_workspace_size(sh, moe.WS_EXPERT_MLP_BF16_DECODE)
+    auto = moe.moe_workspace_size(sh, moe.WS_EXPERT_MLP)
+    assert auto == bs and bs > bf >= 256
+    pre = moe.make_shape(8192, 32, 4, 2880, 2880)  # token-heavy: auto = bf16 decode
+    assert moe.moe_workspace_size(pre, moe.WS_EXPERT_MLP) == \
+        moe.moe_workspace_size(pre, moe.WS_EXPERT_MLP_BF16_DECODE)
+    # (x_perm, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, y_perm, ws, ws_bytes, path, fail, stream)
+    for bad_path in (-1, 3, 99):
+        assert L.moe_expert_mlp_ex(16, 16, sh, 32, 16, 32, 16, 16, 16, 256, bs, bad_path, -1,
+                                   None) == moe.MOE_ERR_INVALID_ARG
+    # a workspace that fits one path is too small for the other
+    assert L.moe_expert_mlp_ex(16, 16, sh, 32, 16, 32, 16, 16, 16, 256, bf,
+                               moe.MOE_MLP_PATH_BLOCK_SCALED, -1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_expert_mlp_ex(16, 16, sh, 32, 16, 32, 16, None, 16, 256, bs,
+                               moe.MOE_MLP_PATH_BF16_DECODE, -1, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_mlp_ex(16, 16, moe.make_shape(64, 32, 4, 2880, 2890), 32, 16, 32, 16, 16,
+                               16, 256, bs, 0, -1, None) == moe.MOE_ERR_SHAPE
 
 
 def test_router_arguments_rejected_before_the_device():
@@ -160,6 +185,11 @@ def test_well_formed_calls_fail_cleanly_without_a_device():
     assert L.moe_expert_mlp(16, 16, sh, 32, 16, 32, 16, 16, 16, 256, mlp, None) in no_device
     assert L.moe_combine(16, 16, 16, sh, 16, None) in no_device
     assert L.moe_layer_forward(16, 16, sh, 32, 16, 32, 16, 16, 256, need, None) in no_device
+    for path in (moe.MOE_MLP_PATH_BLOCK_SCALED, moe.MOE_MLP_PATH_BF16_DECODE):
+        assert L.moe_expert_mlp_ex(16, 16, sh, 32, 16, 32, 16, 16, 16, 256, 1 << 30, path, -1,
+                                   None) in no_device
+    assert L.moe_layer_forward_static(16, 16, sh, 32, 16, 32, 16, 16, None) in no_device
+    assert L.moe_layer_static_status(16, None) in no_device
 
 
 def test_binding_refuses_host_and_strided_tensors():

@@ -1,7 +1,8 @@
 """The expert-parallel layer on the CUDA library with one NCCL rank: the
-exchange degenerates to copies, and the output must equal the one-GPU layer
-bit for bit (the rows reach the grouped GEMM in the same expert groups and
-the same order, and every kernel is deterministic).  The several-rank
+exchange degenerates to copies; the output must meet the layer tolerance
+against the oracle and equal the one-GPU layer bit for bit (the rows reach
+the grouped GEMM in the same expert groups and the same order, and every
+kernel is deterministic).  The several-rank
 exchange is covered on CPU ranks in ``test_ep_gloo.py``; agentlenshq
 "Transformers ... GPT-OSS" (ja), section "Expert parallel (EP)"."""
 import datetime
@@ -12,7 +13,9 @@ import torch
 import torch.distributed as dist
 
 import mxfp4_quantised_mixture_b200 as moe
+import oracle
 import synthetic as syn
+from layer_cases import assert_layer_close, bf16_np, oracle_layer_with_y, oracle_weights_for
 from mxfp4_quantised_mixture_b200 import ep
 
 pytestmark = pytest.mark.gpu
@@ -36,8 +39,9 @@ def test_one_rank_ep_equals_layer(nccl_one_rank, name):
     def bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
 
-    x = bf16(syn.activations(wl))
-    logits = torch.from_numpy(syn.logits(wl)).to(dev)
+    x_np, lg_np = syn.activations(wl), syn.logits(wl)
+    x = bf16(x_np)
+    logits = torch.from_numpy(lg_np).to(dev)
     wgu_q = torch.empty((E, 2 * F, D // 2), dtype=torch.uint8, device=dev)
     wgu_s = torch.empty((E, 2 * F, D // 32), dtype=torch.uint8, device=dev)
     wdn_q = torch.empty((E, D, F // 2), dtype=torch.uint8, device=dev)
@@ -55,3 +59,7 @@ def test_one_rank_ep_equals_layer(nccl_one_rank, name):
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    # and against the oracle's one-process layer
+    gq, gs, dq, ds = oracle_weights_for(wl, range(E))
+    want, y_ulp = oracle_layer_with_y(x_np, lg_np, k, gq, gs, dq, ds)
+    assert_layer_close(bf16_np(out), want, f"ep {name}", y_ulp)
