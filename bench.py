@@ -88,6 +88,8 @@ def parse():
                     help="time this workload alone (default: the headline and all others)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="with --workload: only the warm-up and timed layer steps (for profilers)")
     return ap.parse_args()
 
 
@@ -418,8 +420,9 @@ def quantised_weights(moe, ctx, wl, keep_first_chunk=False, keep_bf16=False):
                                           "bf16": (bf_gu, bf_dn) if keep_bf16 else None}
 
 
-def measure_workload(moe, ctx, wl, weights) -> dict:
-    """Time one workload: the layer step, the expert MLP's roofline, e2e."""
+def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
+    """Time one workload: the layer step, the expert MLP's roofline, e2e
+    (with layer_only, the layer step alone)."""
     import torch
 
     args, dev, stream, flush = ctx.args, ctx.dev, ctx.stream, ctx.flush
@@ -468,6 +471,10 @@ def measure_workload(moe, ctx, wl, weights) -> dict:
     total_ms = reduce_max(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(ctx.world, T, args.steps, total_ms)
+    if layer_only:
+        return {"value": value, "ms_per_step": ms_per_step, "config": config_dict(wl),
+                "clocks": clk, "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
+                "step_ms_min": min(step_ms), "step_ms_max": max(step_ms)}
 
     # ---- roofline of the grouped expert MLP: the same step through the
     #      individual calls, with events around moe_expert_mlp
@@ -649,6 +656,19 @@ def run_ours(args):
     import mxfp4_quantised_mixture_b200 as moe
 
     ctx = Ctx(args)
+    if args.layer_only:
+        if not args.workload:
+            raise SystemExit("--layer-only needs --workload")
+        wl = syn.WORKLOADS[args.workload]
+        weights, _ = quantised_weights(moe, ctx, wl)
+        r = measure_workload(moe, ctx, wl, weights, layer_only=True)
+        if ctx.world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if ctx.rank == 0:
+            print(json.dumps(dict(r, metric=METRIC, unit=UNIT, n_gpus=ctx.world, steps=args.steps,
+                                  warmup=args.warmup, layer_only=True)), flush=True)
+        return 0
     names = [args.workload] if args.workload else [HEADLINE] + OTHERS
     results = {}
     extras = {}

@@ -242,11 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rows_per_expert = args.rows_per_expert, K = args.K, NS = args.NS, NB = args.NB;
   const Tile* __restrict__ tiles = args.tiles;
   int32_t* status = args.status;
-  const int n_tiles = __ldg(args.n_tiles);
   const int F = rows_per_expert / 2;
   const int n_mt = GATE_UP ? (F + BN / 2 - 1) / (BN / 2) : (rows_per_expert + BN - 1) / BN;
-  const int n_items = n_tiles * n_mt;
-  if (static_cast<int>(blockIdx.x) >= n_items) return;  // whole CTA, before any set-up
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -305,6 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t t_sf = tmem + 2 * BN;  // stage slot s: columns t_sf + s * kSlotCols ...
   int my_stages = 0;  // scale writers: stages this warp has arrived on
+  // everything above is independent of the inputs; from here on the previous
+  // kernel's results are needed (a CTA with no item runs no role loop and
+  // goes straight to the unwind)
+  wait_previous_kernel();
+  allow_next_kernel();
+  const int n_items = __ldg(args.n_tiles) * n_mt;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -710,6 +713,8 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
     const uint16_t* __restrict__ src, const int32_t* __restrict__ gather, int k, int K,
     const Tile* __restrict__ tiles, const int* __restrict__ n_tiles, int NT, int64_t padded_rows,
     uint8_t* __restrict__ pieces, uint32_t* __restrict__ words) {
+  wait_previous_kernel();
+  allow_next_kernel();
   const int nstg = (K + BKS - 1) / BKS;
   const int st = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -884,8 +889,8 @@ moe_status launch_gemm(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap
   // each CTA holds all 512 tensor-memory columns: ask for enough shared
   // memory that no second CTA shares the SM
   const int smem_launch = smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
-  grouped_mx_gemm<NT, GATE_UP><<<grid, kThreads, smem_launch, stream>>>(mw, mwt, mx, a);
-  return launch_status();
+  return launch(grouped_mx_gemm<NT, GATE_UP>, dim3(grid), dim3(kThreads), smem_launch, stream,
+                true, mw, mwt, mx, a);
 }
 
 template <bool GATE_UP>
@@ -976,10 +981,13 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
     const bool from_x = in.x != nullptr;
     const int nwin = (D + BKS - 1) / BKS;
     const int64_t blocks = (P.padded_rows + 7) / 8;  // 8 warps per block, one row each
-    split_rows_kernel<<<dim3(static_cast<unsigned>(blocks), nwin), 256, 0, stream>>>(
-        from_x ? in.x : p.x_perm, from_x ? in.sorted_slot : nullptr, from_x ? in.k : 1, D,
-        p.tiles, p.n_tiles, NT, P.padded_rows, P.pieces_x, P.words_x);
-    if ((st = launch_status()) != MOE_OK) return st;
+    // after the tile plan, or after the layer's permute
+    st = launch(split_rows_kernel, dim3(static_cast<unsigned>(blocks), nwin), dim3(256), 0, stream,
+                in.overlap || !in.tiles_ready, from_x ? in.x : p.x_perm,
+                from_x ? in.sorted_slot : static_cast<const int32_t*>(nullptr), from_x ? in.k : 1,
+                D, static_cast<const Tile*>(p.tiles), static_cast<const int*>(p.n_tiles), NT,
+                P.padded_rows, P.pieces_x, P.words_x);
+    if (st != MOE_OK) return st;
   }
   const int max_tiles = static_cast<int>(P.max_tiles);
   const int mt_gu = (F + BN / 2 - 1) / (BN / 2), mt_dn = (D + BN - 1) / BN;
