@@ -191,9 +191,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // [d0, d0 + 128) (one range); both clipped to the matrix.
 template <bool GATE_UP>
 __device__ __forceinline__ void prefetch_item(const uint8_t* wq, const Tile* tiles, int i,
-                                              int n_mt, int rows_per_expert, int K) {
+                                              int n_mt, int rows_per_expert, int K, int E) {
   const int t = i / n_mt, mt = i % n_mt;
-  const int e = __ldg(&tiles[t].e);
+  const int e = min(max(__ldcg(&tiles[t].e), 0), E - 1);
   const int64_t row_bytes = K / 2;
   const uint8_t* base = wq + static_cast<int64_t>(e) * rows_per_expert * row_bytes;
   auto range = [&](int64_t r0, int rows) {
@@ -220,6 +220,7 @@ struct GemmArgs {
   const uint8_t* wq;          // weight codes [E][R][K/2] (for the L2 prefetch)
   const Tile* tiles;
   const int* n_tiles;
+  int max_tiles, E;  // bounds of the tile list and of the expert index
   int rows_per_expert, K, NS, NB, out_ld;
   uint16_t* out;  // h (gate/up; may be null) or y_perm (down)
   // gate/up only: the pieces of h for the down GEMM, [2 * padded rows][F]
@@ -302,6 +303,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t t_sf = tmem + 2 * BN;  // stage slot s: columns t_sf + s * kSlotCols ...
   int my_stages = 0;  // scale writers: stages this warp has arrived on
+  if (warp == 0 && lane == 0) {
+    // Before waiting for the previous kernel: ask L2 for this CTA's first
+    // item's weight rows.  The tile list comes from a kernel at least two
+    // launches back (the permute or the tile plan, then the split or the
+    // gate/up GEMM), which has completed by the time this CTA runs; the
+    // indices are clamped all the same, and a prefetch changes no result.
+    const int nt = min(max(__ldcg(args.n_tiles), 0), args.max_tiles);
+    if (static_cast<int>(blockIdx.x) < nt * n_mt)
+      prefetch_item<GATE_UP>(args.wq, tiles, blockIdx.x, n_mt, rows_per_expert, K, args.E);
+  }
   // everything above is independent of the inputs; from here on the previous
   // kernel's results are needed (a CTA with no item runs no role loop and
   // goes straight to the unwind)
@@ -321,9 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile tile = tiles[t];
         // this item's rows were prefetched with the previous item (the first
         // item's now); ask for the next item's
-        if (it == 0) prefetch_item<GATE_UP>(args.wq, tiles, i, n_mt, rows_per_expert, K);
+        if (it == 0) prefetch_item<GATE_UP>(args.wq, tiles, i, n_mt, rows_per_expert, K, args.E);
         if (i + static_cast<int>(gridDim.x) < n_items)
-          prefetch_item<GATE_UP>(args.wq, tiles, i + gridDim.x, n_mt, rows_per_expert, K);
+          prefetch_item<GATE_UP>(args.wq, tiles, i + gridDim.x, n_mt, rows_per_expert, K, args.E);
         const int b = it % NB, use = it / NB;
         // the auxiliary buffer is free once the scale writers are done with its last item
         if (use > 0 && !wait1(&sfree[b], (use - 1) & 1, abort_flag, status)) break;
@@ -994,6 +1005,8 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
   GemmArgs a{};
   a.tiles = p.tiles;
   a.n_tiles = p.n_tiles;
+  a.max_tiles = max_tiles;
+  a.E = E;
   a.NS = P.NS;
   a.NB = P.NB;
   a.status = status;
