@@ -41,10 +41,11 @@
 // 128-K windows each, so one barrier round trip covers 256 of K) runs on
 // across items, the weight-scale block of an item is double-buffered and so
 // is the accumulator, so one item's epilogue overlaps the next item's MMAs.
-// When an item starts, the producer asks L2 to prefetch the CTA's next
-// item's weight rows (contiguous ranges of the codes), so the ring's copies
-// of that item meet L2 rather than HBM latency while the prefetch keeps more
-// bytes in flight than the ring's shared memory could.
+// With every weight window it loads, the producer asks L2 to prefetch the
+// same window of the CTA's next item (a tensor prefetch with the same map),
+// so the ring's copies of that item meet L2 rather than HBM latency while the
+// prefetches keep more bytes in flight than the ring's shared memory could;
+// the first item's rows are prefetched before the ring starts.
 // Warp roles (14 warps):
 //   warp 0      producer: per item the weight-scale bytes and the token-scale
 //               words (bulk copies), per 128-K window the weight codes (TMA,
@@ -330,11 +331,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
         const int t = i / n_mt, mt = i % n_mt;
         const Tile tile = tiles[t];
-        // this item's rows were prefetched with the previous item (the first
-        // item's now); ask for the next item's
-        if (it == 0) prefetch_item<GATE_UP>(args.wq, tiles, i, n_mt, rows_per_expert, K, args.E);
-        if (i + static_cast<int>(gridDim.x) < n_items)
-          prefetch_item<GATE_UP>(args.wq, tiles, i + gridDim.x, n_mt, rows_per_expert, K, args.E);
+        // the next item of this CTA: with every window this item's ring
+        // loads, L2 is asked for the same window of the next item's weight
+        // rows, so the prefetches run one item ahead at the rate the ring
+        // consumes (the first item was prefetched before the ring started)
+        const int inext = i + static_cast<int>(gridDim.x);
+        const bool has_next = inext < n_items;
+        int next_e = 0, next_wrow = 0;
+        if (has_next) {
+          const int mtn = inext % n_mt;
+          next_e = tiles[inext / n_mt].e;
+          next_wrow = GATE_UP ? mtn * (BN / 2) : mtn * BN;
+        }
         const int b = it % NB, use = it / NB;
         // the auxiliary buffer is free once the scale writers are done with its last item
         if (use > 0 && !wait1(&sfree[b], (use - 1) & 1, abort_flag, status)) break;
@@ -370,15 +378,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int k0 = stage_k0(w, K);
             uint8_t* wdst = wsm + (s_slot * WPS + v) * W_SMEM;
             if (k0 == w * BKS) {
-              if (GATE_UP)
+              if (GATE_UP) {
                 tc::tma_load_5d(wdst, &map_w, &full[s_slot], 0, w, 0, wrow, tile.e);
-              else
+                if (has_next) tc::tma_prefetch_l2_5d(&map_w, 0, w, 0, next_wrow, next_e);
+              } else {
                 tc::tma_load_4d(wdst, &map_w, &full[s_slot], 0, w, wrow, tile.e);
+                if (has_next) tc::tma_prefetch_l2_4d(&map_w, 0, w, next_wrow, next_e);
+              }
             } else {
-              if (GATE_UP)
+              if (GATE_UP) {
                 tc::tma_load_4d(wdst, &map_w_tail, &full[s_slot], 0, 0, wrow, tile.e);
-              else
+                if (has_next) tc::tma_prefetch_l2_4d(&map_w_tail, 0, 0, next_wrow, next_e);
+              } else {
                 tc::tma_load_3d(wdst, &map_w_tail, &full[s_slot], 0, wrow, tile.e);
+                if (has_next) tc::tma_prefetch_l2_3d(&map_w_tail, 0, next_wrow, next_e);
+              }
             }
             tc::tma_load_2d(xs + (s_slot * WPS + v) * X_BYTES, &map_x, &full[s_slot], k0, t * XR);
           }

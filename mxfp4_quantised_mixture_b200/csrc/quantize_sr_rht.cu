@@ -149,8 +149,9 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
     uint32_t out[4];
     int sb = 0;
     bool nonfinite = false;
-    if (srq::block_fits_f32<RHT>(xf)) {
-      // fp32 holds every value of this block exactly (nearly every block)
+    // one path per warp (a warp split between the two would run both): fp32
+    // when it holds every value of all 32 of the warp's blocks exactly
+    if (__all_sync(0xFFFFFFFFu, srq::block_fits_f32<RHT>(xf))) {
       srq::encode_block_f32<RHT, SR>(xf, words, out, sb, nonfinite);
     } else {
       // fp64: the exact widening (subnormals included; Inf and NaN stay

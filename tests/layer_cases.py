@@ -151,6 +151,30 @@ def oracle_layer_with_y(x, lg, k, gq, gs, dq, ds):
     return out, bf16_ulp(yt).max(axis=1)
 
 
+def h_flip_bound(h_bits, offsets, w_dn) -> np.ndarray:
+    """Per element of y [S][D]: how far one bf16 h value rounded to its other
+    neighbour moves it, max_n |w_dn[e][d][n]| * ulp(h[r][n]) with e the
+    expert of row r (bounded by max_n |w| times max_n ulp(h)).  h is a
+    rounding point of the method: where the library (fp32 accumulation) and
+    the oracle (fp64) see g or u within fp32 error of a bf16 rounding
+    boundary, their h differ by one ulp, and y = h . w_dn^T carries it.
+    w_dn: the down weights as values, [E][D][F] (decoded MXFP4 or bf16)."""
+    S, F = h_bits.shape
+    hul = bf16_ulp(h_bits).max(axis=1) if S else np.zeros(0)
+    out = np.zeros((S, w_dn.shape[1]))
+    for e in range(len(offsets) - 1):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 > r0:
+            wmax = np.abs(w_dn[e]).max(axis=1)
+            out[r0:r1] = hul[r0:r1, None] * wmax[None, :]
+    return out
+
+
+def decoded_down(dq, ds) -> np.ndarray:
+    """The oracle's decoded down weights [E][D][F] (fp64)."""
+    return oracle.mxfp4_decode(dq, ds)
+
+
 def oracle_tokens_with_y(x, lg, k, gq, gs, dq, ds, tokens):
     out, y = oracle.layer_tokens(x, lg, k, gq, gs, dq, ds, tokens, want_y=True)
     return out, bf16_ulp(y).max(axis=1)
