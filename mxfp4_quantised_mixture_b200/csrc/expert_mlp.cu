@@ -41,11 +41,6 @@
 // 128-K windows each, so one barrier round trip covers 256 of K) runs on
 // across items, the weight-scale block of an item is double-buffered and so
 // is the accumulator, so one item's epilogue overlaps the next item's MMAs.
-// With every weight window it loads, the producer asks L2 to prefetch the
-// same window of the CTA's next item (a tensor prefetch with the same map),
-// so the ring's copies of that item meet L2 rather than HBM latency while the
-// prefetches keep more bytes in flight than the ring's shared memory could;
-// the first item's rows are prefetched before the ring starts.
 // Warp roles (14 warps):
 //   warp 0      producer: per item the weight-scale bytes and the token-scale
 //               words (bulk copies), per 128-K window the weight codes (TMA,
@@ -99,7 +94,6 @@ constexpr int kSlotCols = 8 * WPS;  // per stage and window: 4 token-scale + 4 w
 constexpr int kTmemCols = 512;      // two accumulators of BN columns, then the scale slots
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestWaitNs = 200000ull;  // the injected wait of test_timeout_cta
-constexpr uint32_t kPrefetchChunk = 32768;   // bytes per L2 prefetch instruction
 
 // Per work item the producer also loads an auxiliary block: the weight-scale
 // bytes of the item's rows [BN][K/32] and the token-scale words of its tile
@@ -187,41 +181,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return r;
 }
 
-// Ask L2 for the weight rows of work item i: gate/up, rows [f0, f0 + 64) of
-// the gate and of the up half (two contiguous ranges); down, rows
-// [d0, d0 + 128) (one range); both clipped to the matrix.
-template <bool GATE_UP>
-__device__ __forceinline__ void prefetch_item(const uint8_t* wq, const Tile* tiles, int i,
-                                              int n_mt, int rows_per_expert, int K, int E) {
-  const int t = i / n_mt, mt = i % n_mt;
-  const int e = min(max(__ldcg(&tiles[t].e), 0), E - 1);
-  const int64_t row_bytes = K / 2;
-  const uint8_t* base = wq + static_cast<int64_t>(e) * rows_per_expert * row_bytes;
-  auto range = [&](int64_t r0, int rows) {
-    const uint8_t* p = base + r0 * row_bytes;
-    const uint32_t bytes = static_cast<uint32_t>(rows * row_bytes);
-    for (uint32_t o = 0; o < bytes; o += kPrefetchChunk)
-      tc::prefetch_l2(p + o, min(kPrefetchChunk, bytes - o));
-  };
-  if (GATE_UP) {
-    const int F = rows_per_expert / 2, f0 = mt * (BN / 2);
-    const int rows = min(BN / 2, F - f0);
-    range(f0, rows);
-    range(F + f0, rows);
-  } else {
-    const int d0 = mt * BN;
-    range(d0, min(BN, rows_per_expert - d0));
-  }
-}
-
 // Arguments of one GEMM launch.
 struct GemmArgs {
   const uint32_t* sfx_words;  // token-scale words of the input pieces
   const uint8_t* scales;      // weight scale bytes [E][R][K/32]
-  const uint8_t* wq;          // weight codes [E][R][K/2] (for the L2 prefetch)
   const Tile* tiles;
   const int* n_tiles;
-  int max_tiles, E;  // bounds of the tile list and of the expert index
   int rows_per_expert, K, NS, NB, out_ld;
   uint16_t* out;  // h (gate/up; may be null) or y_perm (down)
   // gate/up only: the pieces of h for the down GEMM, [2 * padded rows][F]
@@ -304,16 +269,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t t_sf = tmem + 2 * BN;  // stage slot s: columns t_sf + s * kSlotCols ...
   int my_stages = 0;  // scale writers: stages this warp has arrived on
-  if (warp == 0 && lane == 0) {
-    // Before waiting for the previous kernel: ask L2 for this CTA's first
-    // item's weight rows.  The tile list comes from a kernel at least two
-    // launches back (the permute or the tile plan, then the split or the
-    // gate/up GEMM), which has completed by the time this CTA runs; the
-    // indices are clamped all the same, and a prefetch changes no result.
-    const int nt = min(max(__ldcg(args.n_tiles), 0), args.max_tiles);
-    if (static_cast<int>(blockIdx.x) < nt * n_mt)
-      prefetch_item<GATE_UP>(args.wq, tiles, blockIdx.x, n_mt, rows_per_expert, K, args.E);
-  }
   // everything above is independent of the inputs; from here on the previous
   // kernel's results are needed (a CTA with no item runs no role loop and
   // goes straight to the unwind)
@@ -331,18 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
         const int t = i / n_mt, mt = i % n_mt;
         const Tile tile = tiles[t];
-        // the next item of this CTA: with every window this item's ring
-        // loads, L2 is asked for the same window of the next item's weight
-        // rows, so the prefetches run one item ahead at the rate the ring
-        // consumes (the first item was prefetched before the ring started)
-        const int inext = i + static_cast<int>(gridDim.x);
-        const bool has_next = inext < n_items;
-        int next_e = 0, next_wrow = 0;
-        if (has_next) {
-          const int mtn = inext % n_mt;
-          next_e = tiles[inext / n_mt].e;
-          next_wrow = GATE_UP ? mtn * (BN / 2) : mtn * BN;
-        }
         const int b = it % NB, use = it / NB;
         // the auxiliary buffer is free once the scale writers are done with its last item
         if (use > 0 && !wait1(&sfree[b], (use - 1) & 1, abort_flag, status)) break;
@@ -380,18 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k0 == w * BKS) {
               if (GATE_UP) {
                 tc::tma_load_5d(wdst, &map_w, &full[s_slot], 0, w, 0, wrow, tile.e);
-                if (has_next) tc::tma_prefetch_l2_5d(&map_w, 0, w, 0, next_wrow, next_e);
               } else {
                 tc::tma_load_4d(wdst, &map_w, &full[s_slot], 0, w, wrow, tile.e);
-                if (has_next) tc::tma_prefetch_l2_4d(&map_w, 0, w, next_wrow, next_e);
               }
             } else {
               if (GATE_UP) {
                 tc::tma_load_4d(wdst, &map_w_tail, &full[s_slot], 0, 0, wrow, tile.e);
-                if (has_next) tc::tma_prefetch_l2_4d(&map_w_tail, 0, 0, next_wrow, next_e);
               } else {
                 tc::tma_load_3d(wdst, &map_w_tail, &full[s_slot], 0, wrow, tile.e);
-                if (has_next) tc::tma_prefetch_l2_3d(&map_w_tail, 0, next_wrow, next_e);
               }
             }
             tc::tma_load_2d(xs + (s_slot * WPS + v) * X_BYTES, &map_x, &full[s_slot], k0, t * XR);
@@ -1019,15 +958,12 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
   GemmArgs a{};
   a.tiles = p.tiles;
   a.n_tiles = p.n_tiles;
-  a.max_tiles = max_tiles;
-  a.E = E;
   a.NS = P.NS;
   a.NB = P.NB;
   a.status = status;
   // gate/up + SwiGLU: h (when asked) and the pieces of h
   a.sfx_words = P.words_x;
   a.scales = p.wgu_s;
-  a.wq = p.wgu_q;
   a.rows_per_expert = 2 * F;
   a.K = D;
   a.out_ld = F;
@@ -1040,7 +976,6 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
   // down
   a.sfx_words = P.words_h;
   a.scales = p.wdn_s;
-  a.wq = p.wdn_q;
   a.rows_per_expert = D;
   a.K = F;
   a.out_ld = D;

@@ -33,7 +33,6 @@
 // The fp64 butterfly, Philox and the integer encoding make the kernel
 // instruction-bound rather than HBM-bound.
 #include "common.cuh"
-#include "quantize_sr_rht_f32.cuh"
 
 namespace moe {
 namespace {
@@ -124,97 +123,81 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
     const bool valid = blk < nblocks;
     const uint32_t sgn = (RHT && valid) ? __ldg(signs + col) : 0u;
 
-    // bf16 -> fp32 bit pattern (a shift), with the sign flip of the
-    // transform on its sign bit
-    uint32_t xf[32];
+    // bf16 -> fp32 bit pattern (a shift), the sign flip of the transform on
+    // its sign bit, then the exact widening to fp64 (subnormals included;
+    // Inf and NaN stay non-finite and are caught through the block maximum)
+    double y[32];
 #pragma unroll
     for (int t = 0; t < 32; ++t) {
       const uint32_t wd = word[t >> 1];
       uint32_t f = (t & 1) ? (wd & 0xFFFF0000u) : (wd << 16);
       if (RHT) f ^= (sgn << (31 - t)) & 0x80000000u;
-      xf[t] = f;
+      y[t] = static_cast<double>(__uint_as_float(f));
     }
-    // the uniforms of element group g: one Philox4x32-10 output per 8 elements
-    auto words = [&](int g, uint32_t(&rw)[4]) {
-      const uint64_t ctr = static_cast<uint64_t>(blk) * 4 + g;  // (32 blk + 8 g) / 8
-      const uint4 rnd = philox4x32_10(
-          make_uint4(static_cast<uint32_t>(ctr), static_cast<uint32_t>(ctr >> 32), 0u, 0u), key0,
-          key1);
-      rw[0] = rnd.x;
-      rw[1] = rnd.y;
-      rw[2] = rnd.z;
-      rw[3] = rnd.w;
-    };
+    if (RHT) {
+      // in-place fast Walsh-Hadamard transform, natural (Sylvester) order
+#pragma unroll
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if ((i & h) == 0) {
+            const double a = y[i], c = y[i + h];
+            y[i] = a + c;
+            y[i + h] = a - c;
+          }
+        }
+      }
+    }
+
+    // block maximum of |y| through the high words (magnitude order), then
+    // the significand test of the stochastic-rounding scale rule
+    uint32_t amax_hi = 0;
+#pragma unroll
+    for (int t = 0; t < 32; ++t)
+      amax_hi = max(amax_hi, static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu);
+    const bool nonfinite = amax_hi >= 0x7FF00000u;  // an Inf or NaN reached y
+    int sb = 0;
+    if (amax_hi != 0) {
+      sb = static_cast<int>(amax_hi >> 20) - 1023 + 125;
+      if (SR) {
+        const uint32_t frac_hi = amax_hi & 0xFFFFFu;
+        bool above = frac_hi > 0x80000u;
+        if (frac_hi == 0x80000u) {  // significand 1.5 in the high word: the low words decide
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            above |= (static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu) == amax_hi &&
+                     __double2loint(y[t]) != 0;
+        }
+        sb += above ? 1 : 0;
+      }
+      sb = min(max(sb, 0), 254);
+    }
+    const double inv_scale = __hiloint2double((127 - sb + 1023) << 20, 0);  // 2^(127 - sb)
 
     uint32_t out[4];
-    int sb = 0;
-    bool nonfinite = false;
-    // one path per warp (a warp split between the two would run both): fp32
-    // when it holds every value of all 32 of the warp's blocks exactly
-    if (__all_sync(0xFFFFFFFFu, srq::block_fits_f32<RHT>(xf))) {
-      srq::encode_block_f32<RHT, SR>(xf, words, out, sb, nonfinite);
-    } else {
-      // fp64: the exact widening (subnormals included; Inf and NaN stay
-      // non-finite and are caught through the block maximum)
-      double y[32];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) y[t] = static_cast<double>(__uint_as_float(xf[t]));
-      if (RHT) {
-        // in-place fast Walsh-Hadamard transform, natural (Sylvester) order
-#pragma unroll
-        for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if ((i & h) == 0) {
-              const double a = y[i], c = y[i + h];
-              y[i] = a + c;
-              y[i + h] = a - c;
-            }
-          }
-        }
+    for (int g = 0; g < 4; ++g) {
+      uint4 rnd = make_uint4(0u, 0u, 0u, 0u);
+      if (SR) {
+        const uint64_t ctr = static_cast<uint64_t>(blk) * 4 + g;  // (32 blk + 8 g) / 8
+        rnd = philox4x32_10(make_uint4(static_cast<uint32_t>(ctr), static_cast<uint32_t>(ctr >> 32),
+                                       0u, 0u),
+                            key0, key1);
       }
-
-      // block maximum of |y| through the high words (magnitude order), then
-      // the significand test of the stochastic-rounding scale rule
-      uint32_t amax_hi = 0;
+      const uint32_t rw[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+      uint32_t o = 0;
 #pragma unroll
-      for (int t = 0; t < 32; ++t)
-        amax_hi = max(amax_hi, static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu);
-      nonfinite = amax_hi >= 0x7FF00000u;  // an Inf or NaN reached y
-      if (amax_hi != 0) {
-        sb = static_cast<int>(amax_hi >> 20) - 1023 + 125;
-        if (SR) {
-          const uint32_t frac_hi = amax_hi & 0xFFFFFu;
-          bool above = frac_hi > 0x80000u;
-          if (frac_hi == 0x80000u) {  // significand 1.5 in the high word: the low words decide
-#pragma unroll
-            for (int t = 0; t < 32; ++t)
-              above |= (static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu) == amax_hi &&
-                       __double2loint(y[t]) != 0;
-          }
-          sb += above ? 1 : 0;
-        }
-        sb = min(max(sb, 0), 254);
+      for (int e = 0; e < 8; ++e) {
+        const int t = 8 * g + e;
+        const uint32_t u = (rw[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+        uint32_t c = e2m1_code<SR>(fabs(y[t]) * inv_scale, u);
+        // sign bit: that of x without the transform (-0 included); with it,
+        // y < 0 only (a high word above 0x80000000 is a negative nonzero)
+        const uint32_t hy = static_cast<uint32_t>(__double2hiint(y[t]));
+        c |= (RHT ? (hy > 0x80000000u ? 1u : 0u) : (hy >> 31)) << 3;
+        o |= c << (4 * e);
       }
-      const double inv_scale = __hiloint2double((127 - sb + 1023) << 20, 0);  // 2^(127 - sb)
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t rw[4] = {0u, 0u, 0u, 0u};
-        if (SR) words(g, rw);
-        uint32_t o = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int t = 8 * g + e;
-          const uint32_t u = (rw[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-          uint32_t c = e2m1_code<SR>(fabs(y[t]) * inv_scale, u);
-          // sign bit: that of x without the transform (-0 included); with it,
-          // y < 0 only (a high word above 0x80000000 is a negative nonzero)
-          const uint32_t hy = static_cast<uint32_t>(__double2hiint(y[t]));
-          c |= (RHT ? (hy > 0x80000000u ? 1u : 0u) : (hy >> 31)) << 3;
-          o |= c << (4 * e);
-        }
-        out[g] = o;
-      }
+      out[g] = o;
     }
     if (valid) {
       q[blk] = make_uint4(out[0], out[1], out[2], out[3]);
