@@ -18,9 +18,9 @@ moe_status route_launch(const float* logits, int T, int E, int k, int32_t* idx, 
 moe_status permute_launch(const int32_t* idx, const uint16_t* x, const moe_shape& sh,
                           int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
                           int32_t* slot_pos, uint16_t* x_perm, int NT, Tile* tiles,
-                          int* n_tiles, bool overlap, cudaStream_t stream);
+                          int* n_tiles, cudaStream_t stream);
 moe_status combine_launch(const uint16_t* y_perm, const int32_t* slot_pos, const float* w,
-                          const moe_shape& sh, uint16_t* out, bool overlap, cudaStream_t stream);
+                          const moe_shape& sh, uint16_t* out, cudaStream_t stream);
 size_t unquantised_workspace(const moe_shape& sh);
 moe_status unquantised_mlp(const uint16_t* x_perm, const int32_t* offsets, const moe_shape& sh,
                            const uint16_t* w_gu, const uint16_t* w_dn, uint16_t* h,
@@ -266,20 +266,18 @@ moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape s
   if ((st = route_launch(logits, shape.T, shape.E, shape.k, idx, w, status, s)) != MOE_OK)
     return st;
   if ((st = permute_launch(idx, x, shape, counts, offsets, sorted_slot, slot_pos,
-                           block_scaled ? nullptr : x_perm, NT, plan.tiles, plan.n_tiles, true,
-                           s)) != MOE_OK)
+                           block_scaled ? nullptr : x_perm, NT, plan.tiles, plan.n_tiles, s)) != MOE_OK)
     return st;
   MlpInput in{};
   in.offsets = offsets;
   in.tiles_ready = true;
-  in.overlap = true;  // the MLP's first kernel follows the permute (or the gather)
   if (block_scaled) {
     in.x = x;
     in.sorted_slot = sorted_slot;
     in.k = shape.k;
   }
   if ((st = expert_mlp_enqueue(plan, in, status, -1, s)) != MOE_OK) return st;
-  return combine_launch(y_perm, slot_pos, w, shape, out, true, s);
+  return combine_launch(y_perm, slot_pos, w, shape, out, s);
 }
 
 }  // extern "C"

@@ -21,8 +21,6 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const uint4* __restri
                                                           const float* __restrict__ w, int64_t T,
                                                           int k, int vec_per_row,
                                                           uint4* __restrict__ out) {
-  wait_previous_kernel();
-  allow_next_kernel();
   const int64_t n = T * vec_per_row;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * kThreads) {
@@ -55,14 +53,14 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const uint4* __restri
 }  // namespace
 
 moe_status combine_launch(const uint16_t* y_perm, const int32_t* slot_pos, const float* w,
-                          const moe_shape& sh, uint16_t* out, bool overlap, cudaStream_t stream) {
+                          const moe_shape& sh, uint16_t* out, cudaStream_t stream) {
   if (sh.T == 0) return MOE_OK;
   const int vec = sh.d_model / 8;
   const int64_t n = static_cast<int64_t>(sh.T) * vec;
   int64_t want = (n + kThreads - 1) / kThreads;
   int64_t cap = static_cast<int64_t>(sm_count()) * 16;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  return launch(combine_kernel, dim3(grid), dim3(kThreads), 0, stream, overlap,
+  return launch(combine_kernel, dim3(grid), dim3(kThreads), 0, stream,
                 reinterpret_cast<const uint4*>(y_perm), slot_pos, w, static_cast<int64_t>(sh.T),
                 sh.k, vec, reinterpret_cast<uint4*>(out));
 }
@@ -80,6 +78,5 @@ extern "C" moe_status moe_combine(const uint16_t* y_perm, const int32_t* slot_po
     return MOE_ERR_INVALID_ARG;
   moe_status st = check_device();
   if (st != MOE_OK) return st;
-  return combine_launch(y_perm, slot_pos, topk_w, shape, out, false,
-                        static_cast<cudaStream_t>(stream));
+  return combine_launch(y_perm, slot_pos, topk_w, shape, out, static_cast<cudaStream_t>(stream));
 }

@@ -56,38 +56,20 @@ int sm_count();
 
 bool shape_ok(const moe_shape& s);
 
-// Launch a kernel; with `overlap` as a programmatic dependent of the kernel
-// before it on the stream: it may start while that kernel finishes, runs its
-// data-independent prologue, and waits (griddepcontrol.wait, which every
-// kernel of this library executes before it touches its inputs or exits)
-// until that kernel has completed and its writes are visible.
+// Launch a kernel with cudaLaunchKernelEx (argument coercion as for <<< >>>).
 template <typename... Params, typename... Args>
 moe_status launch(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
-                  cudaStream_t stream, bool overlap, Args&&... args) {
+                  cudaStream_t stream, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = overlap ? attr : nullptr;
-  cfg.numAttrs = overlap ? 1 : 0;
   if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
   return MOE_OK;
-}
-
-// Device side of the above: wait for the previous kernel's completion (a
-// no-op after a normal launch), then let the next kernel start launching.
-__device__ __forceinline__ void wait_previous_kernel() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void allow_next_kernel() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 }  // namespace moe

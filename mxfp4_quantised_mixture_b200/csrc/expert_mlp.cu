@@ -269,11 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t t_sf = tmem + 2 * BN;  // stage slot s: columns t_sf + s * kSlotCols ...
   int my_stages = 0;  // scale writers: stages this warp has arrived on
-  // everything above is independent of the inputs; from here on the previous
-  // kernel's results are needed (a CTA with no item runs no role loop and
-  // goes straight to the unwind)
-  wait_previous_kernel();
-  allow_next_kernel();
+  // a CTA with no item runs no role loop and goes straight to the unwind
   const int n_items = __ldg(args.n_tiles) * n_mt;
 
   if (warp == 0) {
@@ -677,8 +673,6 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
     const uint16_t* __restrict__ src, const int32_t* __restrict__ gather, int k, int K,
     const Tile* __restrict__ tiles, const int* __restrict__ n_tiles, int NT, int64_t padded_rows,
     uint8_t* __restrict__ pieces, uint32_t* __restrict__ words) {
-  wait_previous_kernel();
-  allow_next_kernel();
   const int nstg = (K + BKS - 1) / BKS;
   const int st = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -854,7 +848,7 @@ moe_status launch_gemm(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap
   // memory that no second CTA shares the SM
   const int smem_launch = smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
   return launch(grouped_mx_gemm<NT, GATE_UP>, dim3(grid), dim3(kThreads), smem_launch, stream,
-                true, mw, mwt, mx, a);
+                mw, mwt, mx, a);
 }
 
 template <bool GATE_UP>
@@ -947,7 +941,7 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
     const int64_t blocks = (P.padded_rows + 7) / 8;  // 8 warps per block, one row each
     // after the tile plan, or after the layer's permute
     st = launch(split_rows_kernel, dim3(static_cast<unsigned>(blocks), nwin), dim3(256), 0, stream,
-                in.overlap || !in.tiles_ready, from_x ? in.x : p.x_perm,
+                from_x ? in.x : p.x_perm,
                 from_x ? in.sorted_slot : static_cast<const int32_t*>(nullptr), from_x ? in.k : 1,
                 D, static_cast<const Tile*>(p.tiles), static_cast<const int*>(p.n_tiles), NT,
                 P.padded_rows, P.pieces_x, P.words_x);

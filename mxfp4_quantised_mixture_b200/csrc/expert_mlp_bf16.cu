@@ -160,10 +160,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
   constexpr int X_STAGE = NT * 128;
   constexpr int TMEM_COLS = tmem_cols_for(NT);
   constexpr uint32_t IDESC = tc::idesc_bf16_f32(BM, NT);
-  // the tile count comes from the previous kernel; a CTA beyond it leaves
-  // before any set-up
-  wait_previous_kernel();
-  allow_next_kernel();
+  // a CTA beyond the tile count leaves before any set-up
   if (static_cast<int>(blockIdx.y) >= __ldg(n_tiles)) return;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -543,10 +540,8 @@ moe_status launch_gemm(const CUtensorMap& mw, const CUtensorMap& mx, const uint8
                        int out_ld, uint16_t* out, int32_t* status, int fail_cta,
                        cudaStream_t stream) {
   const int smem = smem_layout(NT, K).total + 1024;
-  // always after another kernel of this library (the tile plan, the permute's
-  // gather or the gate/up GEMM)
   return launch(grouped_mxfp4_gemm<NT, GATE_UP>, dim3(grid_x, grid_y), dim3(kThreads), smem,
-                stream, true, mw, mx, scales, tiles, n_tiles, R, K, out_ld, out, status,
+                stream, mw, mx, scales, tiles, n_tiles, R, K, out_ld, out, status,
                 fail_cta);
 }
 

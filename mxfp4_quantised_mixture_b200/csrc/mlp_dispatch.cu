@@ -17,8 +17,6 @@ __global__ void __launch_bounds__(256) plan_tiles_kernel(const int32_t* __restri
                                                          int NT, Tile* __restrict__ tiles,
                                                          int* __restrict__ n_tiles) {
   __shared__ int base[257];
-  wait_previous_kernel();
-  allow_next_kernel();
   const int e = threadIdx.x;
   int cnt = 0;
   if (e < E) {
@@ -64,7 +62,7 @@ EncodeTiledFn encode_tiled_fn() {
 
 moe_status plan_tiles_launch(const int32_t* offsets, int E, int NT, Tile* tiles, int* n_tiles,
                              cudaStream_t stream) {
-  return launch(plan_tiles_kernel, dim3(1), dim3(256), 0, stream, false, offsets, E, NT, tiles,
+  return launch(plan_tiles_kernel, dim3(1), dim3(256), 0, stream, offsets, E, NT, tiles,
                 n_tiles);
 }
 

@@ -84,8 +84,6 @@ moe_status bf_plan(MlpPlan* p, void* ws);
 struct MlpInput {
   const int32_t* offsets;  // [E+1], device
   bool tiles_ready;        // the tile list was already written (by the permute)
-  bool overlap;            // the first kernel follows another of this library's kernels
-                           // on the stream (a programmatic dependent launch)
   // block-scaled path inside the layer: split the rows straight from x
   // (row r of the permuted order is x[sorted_slot[r] / k]) instead of x_perm
   const uint16_t* x;

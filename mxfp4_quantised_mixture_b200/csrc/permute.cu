@@ -37,8 +37,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int32_t cnt[kWarps][kMaxE];  // per (warp, expert) count, then running position
   __shared__ int32_t off[kMaxE + 1];
   __shared__ int32_t tbase[kMaxE + 1];    // first tile of each expert (tile list only)
-  wait_previous_kernel();
-  allow_next_kernel();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&cnt[0][0])[i] = 0;
   __syncthreads();
@@ -143,8 +141,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                          const int32_t* __restrict__ n_valid,
                                                          int k, int vec_per_row,
                                                          uint4* __restrict__ x_perm) {
-  wait_previous_kernel();
-  allow_next_kernel();
   const int64_t S = *n_valid;
   const int lane = threadIdx.x & 31;
   const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -162,16 +158,16 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 moe_status permute_launch(const int32_t* idx, const uint16_t* x, const moe_shape& sh,
                           int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
                           int32_t* slot_pos, uint16_t* x_perm, int NT, Tile* tiles,
-                          int* n_tiles, bool overlap, cudaStream_t stream) {
+                          int* n_tiles, cudaStream_t stream) {
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
-  moe_status st = launch(permute_kernel, dim3(1), dim3(kThreads), 0, stream, overlap, idx, S,
+  moe_status st = launch(permute_kernel, dim3(1), dim3(kThreads), 0, stream, idx, S,
                          sh.E, counts, offsets, sorted_slot, slot_pos, NT, tiles, n_tiles);
   if (st != MOE_OK || S == 0 || x_perm == nullptr) return st;
   const int vec = sh.d_model / 8;
   int64_t want = (S * 32 + 255) / 256;
   int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  return launch(gather_rows_kernel, dim3(grid), dim3(256), 0, stream, true,
+  return launch(gather_rows_kernel, dim3(grid), dim3(256), 0, stream,
                 reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(sorted_slot),
                 static_cast<const int32_t*>(offsets + sh.E), sh.k, vec,
                 reinterpret_cast<uint4*>(x_perm));
@@ -196,5 +192,5 @@ extern "C" moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x, mo
   moe_status st = check_device();
   if (st != MOE_OK) return st;
   return permute_launch(topk_idx, x, shape, counts, offsets, sorted_slot, slot_pos, x_perm, 0,
-                        nullptr, nullptr, false, static_cast<cudaStream_t>(stream));
+                        nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }

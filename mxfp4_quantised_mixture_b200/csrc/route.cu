@@ -26,8 +26,6 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
                                                         int E, int k, int32_t* __restrict__ idx,
                                                         float* __restrict__ w,
                                                         int32_t* __restrict__ clear_status) {
-  wait_previous_kernel();
-  allow_next_kernel();
   // inside the layer the routing is the first kernel: it resets the layer's
   // device status word, which the later kernels only ever set to an error
   if (clear_status && blockIdx.x == 0 && threadIdx.x == 0) *clear_status = MOE_OK;
@@ -89,7 +87,7 @@ moe_status route_launch(const float* logits, int T, int E, int k, int32_t* idx, 
                         int32_t* clear_status, cudaStream_t stream) {
   if (T == 0) return MOE_OK;
   const int grid = (T + kThreads / 32 - 1) / (kThreads / 32);
-  return launch(route_kernel, dim3(grid), dim3(kThreads), 0, stream, false, logits, T, E, k, idx,
+  return launch(route_kernel, dim3(grid), dim3(kThreads), 0, stream, logits, T, E, k, idx,
                 w, clear_status);
 }
 
