@@ -22,46 +22,45 @@
 // in a bf16 GEMM on decoded weights, and only the fp32 accumulation order
 // differs from a sequential sum.
 //
-// MMA shape: M = 128 token rows (the hi and lo pieces of up to 64 tokens,
-// interleaved: row 2t = hi of token t, row 2t + 1 = lo), N = 128 weight rows,
-// K = 32.  With the weights on N an MMA covers 128 rows x 32 codes and runs at
-// the tensor core's full rate (64 cycles), so a 128-K window of 8 KB of codes
-// costs 256 cycles of MMA, under the ~370 cycles the SM's share of HBM
-// bandwidth needs to deliver it; narrower MMAs are bound by their issue rate.
-// The epilogue adds rows 2t and 2t + 1 (neighbouring lanes).
+// MMA shape: M = 128 weight rows, N = 2 NT token piece rows (the hi and lo
+// pieces of NT tokens, interleaved: piece row 2t = hi of token t, 2t + 1 =
+// lo), K = 32.  The weights take the M side because the block-scaled MMA
+// reads both operands from shared memory and M is fixed at 128: the token
+// side then costs only its real rows, N x 32 bytes per MMA, and an MMA reads
+// 4 KB of codes plus 1-4 KB of pieces.  The epilogue adds accumulator
+// columns 2t and 2t + 1.
 //   * gate/up: the 128 rows are 64 gate rows and the matching 64 up rows,
 //     interleaved by the copy's box order (row 2j = gate j, 2j + 1 = up j), so
-//     a lane holds both halves of SwiGLU.  The epilogue rounds h to bf16
-//     (stored to h [S][F] when asked) and splits it at once into the pieces
-//     the down GEMM reads: each epilogue warp holds one whole 32-feature block
-//     of h for its tokens.
+//     neighbouring lanes hold the two halves of SwiGLU.  The epilogue rounds
+//     h to bf16 into a shared-memory tile [NT][64], then, one warp per
+//     (token, 32-feature block), stores h to [S][F] when asked and splits it
+//     into the pieces the down GEMM reads.
 //   * down: 128 rows of the [D][F] matrix; output y_perm [S][D] bf16.
 // The kernel is persistent: one CTA per SM walks the work items (token tile,
 // weight slice) b, b + grid, ...; its copy ring (up to 12 stages of two
 // 128-K windows each, so one barrier round trip covers 256 of K) runs on
-// across items, the weight-scale block of an item is double-buffered and so
-// is the accumulator, so one item's epilogue overlaps the next item's MMAs.
+// across items, the weight-scale block of an item is single- or
+// double-buffered and the accumulator double-buffered, so one item's
+// epilogue overlaps the next item's MMAs.
 // Warp roles (14 warps):
 //   warp 0      producer: per item the weight-scale bytes and the token-scale
 //               words (bulk copies), per 128-K window the weight codes (TMA,
 //               8 KB of packed codes that land as the 16 KB one-byte-per-code
 //               layout the MMA reads) and the token pieces (TMA, 2 NT x 128 B)
 //   warp 1      tensor-memory owner and MMA issuer: 4 MMAs per window
-//   warps 2-5   scale writers: per window they copy the token scales and the
-//               weight scales (both from the item's auxiliary block) into the
+//   warps 2-5   scale writers: per window they copy the weight scales and the
+//               token scales (both from the item's auxiliary block) into the
 //               stage slot's scale columns in tensor memory, every lane quarter
 //               its own copy, and add their arrival to the stage's barrier, so
 //               the MMA thread waits on one barrier per stage
-//   warps 6-13  epilogue: two warps per lane quarter, 64 accumulator columns
-//               each; a quarter whose tokens are all padding is skipped
+//   warps 6-13  epilogue: two warps per lane quarter, one per half of the
+//               tile's tokens
 // When K is not a multiple of 128 the last window re-reads [K - 128, K) and
 // issues only the MMAs over its new 32-element blocks.
 // The token pieces sit in a tile-padded layout (tile t owns piece rows
 // [2 t NT, 2 t NT + 2 NT)), so every copy of a tile's rows is aligned and
-// whole; the MMA's 128-row view of a stage narrower than 128 rows reads on
-// into the following shared memory, and those accumulator rows are ignored
-// (an accumulator row depends only on its own operand row and scales, so
-// whatever the padding rows hold never reaches a real token's output).
+// whole.  Pieces of padding rows are never written here (their accumulator
+// columns depend only on their own rows and scales, and are never read).
 // Every wait is bounded (2 s); on expiry the kernel records MOE_ERR_TIMEOUT
 // in the status word and unwinds: every role leaves its loop, the scale
 // writers complete the stage arrivals they skipped (the producer's copy
@@ -83,33 +82,35 @@ namespace {
 
 constexpr int BKS = 128;            // K elements per window (one 128-byte swizzle row of codes)
 constexpr int WPS = 2;              // windows per pipeline stage
-constexpr int BN = 128;             // weight rows per work item (MMA N)
-constexpr int MM = 128;             // MMA M: token piece rows
+constexpr int BN = 128;             // weight rows per work item (MMA M)
 constexpr int W_SMEM = BN * BKS;    // one byte per code in shared memory
 constexpr int W_TX = BN * BKS / 2;  // bytes one window's weight copy reads
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (6 + kEpiWarps);
 constexpr int kMaxStages = 12;      // copy ring depth limit (stage slot s also owns scale slot s)
 constexpr int kSlotCols = 8 * WPS;  // per stage and window: 4 token-scale + 4 weight-scale columns
-constexpr int kTmemCols = 512;      // two accumulators of BN columns, then the scale slots
+constexpr int kAccCols = 128;       // tensor-memory columns per accumulator (N <= 128)
+constexpr int kTmemCols = 512;      // two accumulators, then the scale slots
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestWaitNs = 200000ull;  // the injected wait of test_timeout_cta
 
 // Per work item the producer also loads an auxiliary block: the weight-scale
 // bytes of the item's rows [BN][K/32] and the token-scale words of its tile
 // [stages][2 NT]; NB = 1 or 2 of them (double-buffered across items).
+// The gate/up epilogue also stages h in two tiles [NT][64] bf16.
 struct SmemLayout {
-  int x_off, w_off, a_off, wsc_bytes, aux_bytes, bar_off, total;
+  int x_off, w_off, a_off, wsc_bytes, aux_bytes, h_off, bar_off, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int NT, int NS, int NB, int K) {
   SmemLayout L;
-  L.x_off = 0;  // token ring first: a window's 128-row MMA view runs on into the weight ring
+  L.x_off = 0;
   L.w_off = NS * WPS * 2 * NT * BKS;
   L.a_off = L.w_off + NS * WPS * W_SMEM;
   L.wsc_bytes = ((BN * (K / 32)) + 127) / 128 * 128;
   L.aux_bytes = L.wsc_bytes + ((K + BKS - 1) / BKS) * 2 * NT * 4;
-  L.bar_off = L.a_off + NB * L.aux_bytes;
+  L.h_off = L.a_off + NB * L.aux_bytes;
+  L.bar_off = L.h_off + 2 * NT * (BN / 2) * 2;
   L.total = L.bar_off + 1024;
   return L;
 }
@@ -145,6 +146,15 @@ __device__ __forceinline__ void split4(const float (&v)[4], int t, uint32_t& hi4
     hi4 |= static_cast<uint32_t>(h8) << (8 * j);
     lo4 |= static_cast<uint32_t>(l8) << (8 * j);
   }
+}
+
+// One bf16-exact value -> its hi and lo E4M3 bytes.
+__device__ __forceinline__ void split1(float v, int t, uint8_t& hi, uint8_t& lo) {
+  const float u = v * __uint_as_float(static_cast<uint32_t>(127 - t) << 23);  // v / 2^t
+  const __nv_fp8_storage_t h8 = __nv_cvt_float_to_fp8(u, __NV_SATFINITE, __NV_E4M3);
+  const float hf = __half2float(__half(__nv_cvt_fp8_to_halfraw(h8, __NV_E4M3)));
+  hi = static_cast<uint8_t>(h8);
+  lo = static_cast<uint8_t>(__nv_cvt_float_to_fp8((u - hf) * 16.0f, __NV_SATFINITE, __NV_E4M3));
 }
 
 // ------------------------------------------------------------------ waits
@@ -204,8 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap map_x, const GemmArgs args) {
   constexpr int XR = 2 * NT;  // token piece rows per window
   constexpr uint32_t X_BYTES = XR * BKS;
-  constexpr uint32_t IDESC = tc::idesc_mx(tc::kFmtE4M3, tc::kFmtE2M1, MM, BN);
-  static_assert(XR <= MM && (X_BYTES % 1024) == 0, "token tile of 8..64 tokens");
+  constexpr uint32_t IDESC = tc::idesc_mx(tc::kFmtE2M1, tc::kFmtE4M3, BN, XR);
+  static_assert(XR >= 16 && XR <= kAccCols && (X_BYTES % 1024) == 0, "token tile of 8..64 tokens");
   const int rows_per_expert = args.rows_per_expert, K = args.K, NS = args.NS, NB = args.NB;
   const Tile* __restrict__ tiles = args.tiles;
   int32_t* status = args.status;
@@ -219,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* xs = smem + L.x_off;
   uint8_t* wsm = smem + L.w_off;
   uint8_t* aux = smem + L.a_off;
+  uint16_t* hstage = reinterpret_cast<uint16_t*>(smem + L.h_off);  // [2][NT][64] bf16
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* full = bars;                  // [NS] stage copies landed and scales written
   uint64_t* empty = full + kMaxStages;    // [NS] stage MMAs complete
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t t_sf = tmem + 2 * BN;  // stage slot s: columns t_sf + s * kSlotCols ...
+  const uint32_t t_sf = tmem + 2 * kAccCols;  // stage slot s: columns t_sf + s * kSlotCols ...
   int my_stages = 0;  // scale writers: stages this warp has arrived on
   // a CTA with no item runs no role loop and goes straight to the unwind
   const int n_items = __ldg(args.n_tiles) * n_mt;
@@ -363,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
       }
       for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
-        const uint32_t d = tmem + (it & 1) * BN;
+        const uint32_t d = tmem + (it & 1) * kAccCols;
         // accumulator it & 1 was last used by item it - 2
         if (it >= 2) {
           if (!wait1(&dempty[it & 1], d_phase, abort_flag, status)) break;
@@ -378,20 +389,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::tc_fence_after();
-          // a descriptor addresses shared memory in 16-byte units: +2 per 32 bytes
+          // a descriptor addresses shared memory in 16-byte units: +2 per 32
+          // bytes; A = weights with their scales in the slot's columns 4-7,
+          // B = token pieces with theirs in columns 0-3
 #pragma unroll
           for (int v = 0; v < WPS; ++v) {
             const int w = st * WPS + v;
             if (w >= nwin) break;
             const uint64_t xv = xdesc + v * (X_BYTES >> 4), wv = wdesc + v * (W_SMEM >> 4);
-            const uint32_t sv = sfa + 8 * v;
+            const uint32_t sx = sfa + 8 * v, sw = sx + 4;
             if (w != tail_w) {
-              tc::mma_mx_ss(d, xv, wv, IDESC | tc::idesc_sf_ids(0, 0), w > 0 ? 1u : 0u, sv, sv + 4);
-              tc::mma_mx_ss(d, xv + 2, wv + 2, IDESC | tc::idesc_sf_ids(1, 1), 1u, sv, sv + 4);
+              tc::mma_mx_ss(d, wv, xv, IDESC | tc::idesc_sf_ids(0, 0), w > 0 ? 1u : 0u, sw, sx);
+              tc::mma_mx_ss(d, wv + 2, xv + 2, IDESC | tc::idesc_sf_ids(1, 1), 1u, sw, sx);
             }
-            tc::mma_mx_ss(d, xv + 4, wv + 4, IDESC | tc::idesc_sf_ids(2, 2),
-                          (w != tail_w || w > 0) ? 1u : 0u, sv, sv + 4);
-            tc::mma_mx_ss(d, xv + 6, wv + 6, IDESC | tc::idesc_sf_ids(3, 3), 1u, sv, sv + 4);
+            tc::mma_mx_ss(d, wv + 4, xv + 4, IDESC | tc::idesc_sf_ids(2, 2),
+                          (w != tail_w || w > 0) ? 1u : 0u, sw, sx);
+            tc::mma_mx_ss(d, wv + 6, xv + 6, IDESC | tc::idesc_sf_ids(3, 3), 1u, sw, sx);
           }
           tc::mma_commit(&empty[s_slot]);
           any = true;
@@ -498,101 +511,82 @@ __global__ void __launch_bounds__(kThreads, 1)
     my_stages = g;
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                // tensor-memory lane quarter
-    const int half = (warp - 6) >> 2;      // accumulator columns [64 half, 64 half + 64)
+    // Lane l of quarter q holds weight row m = 32 q + l of the item; this
+    // warp reads the accumulator columns of tokens [half HT, half HT + HT).
+    constexpr int HT = NT / 2;
+    const int q = warp & 3;
+    const int half = (warp - 6) >> 2;
+    const int ew = warp - 6;  // epilogue warp 0..7
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    const int m = q * 32 + lane;  // accumulator row: token m >> 1, piece m & 1
-    const int tl = m >> 1;
-    const bool lo = m & 1;
     int it = 0;
     for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++it) {
       const int t = i / n_mt, mt = i % n_mt;
       const Tile tile = tiles[t];
       const int a = it & 1;
-      if (!warp_wait(&dfull[a], (it >> 1) & 1, abort_flag, status, 256)) break;
-      tc::tc_fence_after();
-      if (16 * q < tile.nrows) {  // this quarter holds at least one real token
-        const bool live_row = tl < tile.nrows;
-        const uint32_t dcol = tmem + a * BN + 64 * half;
-        // 16 accumulator columns starting at item column cc: the hi lane
-        // finishes columns cc..cc+7, the lo lane cc+8..cc+15
-        auto sums16 = [&](const uint32_t(&r)[16], float(&sum)[8]) {
+      const bool ok = warp_wait(&dfull[a], (it >> 1) & 1, abort_flag, status, 256);
+      float acc[HT];  // token half HT + j of this lane's row: hi + lo piece
+      if (ok) {
+        tc::tc_fence_after();
+        const uint32_t dcol = tmem + a * kAccCols + half * NT + lane_base;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float x = __uint_as_float(r[j]);
-            const float y = __uint_as_float(r[8 + j]);
-            const float recv = __shfl_xor_sync(0xFFFFFFFFu, lo ? x : y, 1);
-            sum[j] = (lo ? y : x) + recv;
+        for (int c = 0; c < NT; c += 16) {
+          uint32_t r[16];
+          tc::tmem_ld16(dcol + c, r);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            acc[c / 2 + j] = __uint_as_float(r[2 * j]) + __uint_as_float(r[2 * j + 1]);
+        }
+        // this warp has read its part of the accumulator
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&dempty[a]);
+      }
+      if (GATE_UP) {
+        // lanes 2j (gate) and 2j + 1 (up) hold local feature fl = 16 q + j;
+        // the gate lane finishes the first HT / 2 tokens, the up lane the rest
+        constexpr int QT = HT / 2;
+        const bool up = lane & 1;
+        const int fl = 16 * q + (lane >> 1);
+        uint16_t* hs = hstage + a * NT * (BN / 2);
+        if (ok) {
+#pragma unroll
+          for (int j = 0; j < QT; ++j) {
+            const float recv = __shfl_xor_sync(0xFFFFFFFFu, up ? acc[j] : acc[QT + j], 1);
+            const float gv = up ? recv : acc[j];
+            const float uv = up ? acc[QT + j] : recv;
+            const float hh = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+            hs[(half * HT + (up ? QT : 0) + j) * (BN / 2) + fl] = f32_to_bf16_rne(hh);
           }
-        };
-        if (GATE_UP) {
-          // This warp's 64 columns are the gate/up pairs of one 32-feature
-          // block of h, fb = mt * 64 + 32 * half; the token's two lanes hold
-          // 16 features each: group gi of this lane is features
-          // fb + 8 gi + (lo ? 4 : 0) + 0..3.
-          const int fb = mt * (BN / 2) + 32 * half;
-          float hv[16];
-          uint32_t hb[8];
+        }
+        // every epilogue warp takes part (a failed wait included), so the
+        // barrier cannot strand one; all leave together if any failed
+        if (!tc::bar_and(1, 32 * kEpiWarps, ok)) break;
+        // one warp per (token, 32-feature block): store h, split it into the
+        // pieces of the down GEMM and write the block's scale bytes
+        const int fb0 = mt * (BN / 2);
+        const int nunits = tile.nrows * 2;
+        for (int u = ew; u < nunits; u += kEpiWarps) {
+          const int tl = u >> 1, b = u & 1;
+          const int f = fb0 + 32 * b + lane;
+          const uint16_t hbits = hs[tl * (BN / 2) + 32 * b + lane];
+          const float v = bf16_to_f32(hbits);
+          if (args.out) args.out[static_cast<int64_t>(tile.row0 + tl) * args.out_ld + f] = hbits;
+          float amax = fabsf(v);
 #pragma unroll
-          for (int c = 0; c < 64; c += 32) {
-            uint32_t ra[16], rb[16];
-            tc::tmem_ld16(dcol + lane_base + c, ra);
-            tc::tmem_ld16(dcol + lane_base + c + 16, rb);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              float sum[8];
-              sums16(h2 ? rb : ra, sum);
-              const int gi = (c >> 4) + h2;
-#pragma unroll
-              for (int p2 = 0; p2 < 2; ++p2) {
-                float hh[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  const float gv = sum[4 * p2 + 2 * u], uv = sum[4 * p2 + 2 * u + 1];
-                  hh[u] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-                }
-                const uint32_t w2 = pack_bf16x2(hh[0], hh[1]);
-                hb[2 * gi + p2] = w2;
-                hv[4 * gi + 2 * p2] = __uint_as_float(w2 << 16);
-                hv[4 * gi + 2 * p2 + 1] = __uint_as_float(w2 & 0xFFFF0000u);
-              }
-            }
-          }
-          uint16_t* orow = args.out ? args.out + static_cast<int64_t>(tile.row0 + tl) * args.out_ld
-                                    : nullptr;
-          if (orow && live_row) {
-#pragma unroll
-            for (int gi = 0; gi < 4; ++gi) {
-              const int f = fb + 8 * gi + (lo ? 4 : 0);
-              if (f < F) *reinterpret_cast<uint2*>(orow + f) = make_uint2(hb[2 * gi], hb[2 * gi + 1]);
-            }
-          }
-          // the split of h for the down GEMM: the block's exponent from the
-          // token's 32 features (this lane's 16 and its neighbour's)
-          float amax = 0.f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(hv[j]));
-          amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
           const int te = split_exponent(amax);
+          uint8_t hi, lo;
+          split1(v, te, hi, lo);
           const int64_t p = static_cast<int64_t>(t) * NT + tl;  // padded row of this token
-          uint8_t* prow_hi = args.pieces_out + (2 * p) * F;
-          uint8_t* prow_lo = prow_hi + F;
-#pragma unroll
-          for (int gi = 0; gi < 4; ++gi) {
-            const float v4[4] = {hv[4 * gi], hv[4 * gi + 1], hv[4 * gi + 2], hv[4 * gi + 3]};
-            uint32_t hi4, lo4;
-            split4(v4, te, hi4, lo4);
-            const int f = fb + 8 * gi + (lo ? 4 : 0);
-            *reinterpret_cast<uint32_t*>(prow_hi + f) = hi4;
-            *reinterpret_cast<uint32_t*>(prow_lo + f) = lo4;
-          }
-          if (!lo) {
-            // scale bytes of block fb / 32 in the words of the window(s)
-            // that cover it: window b / 4 (byte b % 4), and, when F is not a
+          args.pieces_out[(2 * p) * F + f] = hi;
+          args.pieces_out[(2 * p + 1) * F + f] = lo;
+          if (lane == 0) {
+            // scale bytes of block blk in the words of the window(s) that
+            // cover it: window blk / 4 (byte blk % 4), and, when F is not a
             // multiple of 128, the moved-back last window [F - 128, F)
             const int nwo = (F + BKS - 1) / BKS;
-            const int blk = fb / 32;
+            const int blk = (fb0 + 32 * b) / 32;
             const int tail0 = (F % BKS) ? (F - BKS) / 32 : 0x7FFFFFFF;
             auto put = [&](int w, int byte) {
               uint8_t* wb = reinterpret_cast<uint8_t*>(
@@ -603,31 +597,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (F % BKS == 0 || blk / 4 < nwo - 1) put(blk / 4, blk % 4);
             if (blk >= tail0) put(nwo - 1, blk - tail0);
           }
-        } else {
-          uint16_t* orow = args.out + static_cast<int64_t>(tile.row0 + tl) * args.out_ld;
-#pragma unroll 1
-          for (int c = 0; c < 64; c += 32) {
-            uint32_t ra[16], rb[16];
-            tc::tmem_ld16(dcol + lane_base + c, ra);
-            tc::tmem_ld16(dcol + lane_base + c + 16, rb);
-            tc::tmem_ld_wait();
+        }
+      } else {
+        if (!ok) break;
+        const int dd = mt * BN + 32 * q + lane;
+        if (dd < rows_per_expert) {
+          uint16_t* ocol = args.out + static_cast<int64_t>(tile.row0) * args.out_ld + dd;
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              float sum[8];
-              sums16(h2 ? rb : ra, sum);
-              const int dd = mt * BN + 64 * half + c + 16 * h2 + (lo ? 8 : 0);
-              if (live_row && dd < rows_per_expert)
-                *reinterpret_cast<uint4*>(orow + dd) =
-                    make_uint4(pack_bf16x2(sum[0], sum[1]), pack_bf16x2(sum[2], sum[3]),
-                               pack_bf16x2(sum[4], sum[5]), pack_bf16x2(sum[6], sum[7]));
-            }
+          for (int j = 0; j < HT; ++j) {
+            const int tl = half * HT + j;
+            if (tl < tile.nrows) ocol[static_cast<int64_t>(tl) * args.out_ld] = f32_to_bf16_rne(acc[j]);
           }
         }
       }
-      // this warp has read its part of the accumulator
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&dempty[a]);
     }
   }
 
@@ -784,8 +766,8 @@ constexpr int kMaxSmemPerCta = 227 * 1024;
 int smem_bytes(int NT, int NS, int NB, int K) { return smem_layout(NT, NS, NB, K).total + 1024; }
 
 // token-tile width: about twice the mean rows per expert, 16..64; then the
-// deepest copy ring (up to 12 stages) beside a double-buffered weight-scale
-// block, with at least 4 stages; failing that, a single scale block
+// deepest copy ring (up to 12 stages), its weight-scale block double-buffered
+// when that costs no stage
 GemmConfig choose_config(const moe_shape& sh) {
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
   const int64_t want = 2 * ((S + sh.E - 1) / sh.E);
@@ -793,10 +775,10 @@ GemmConfig choose_config(const moe_shape& sh) {
   while (nt < want && nt < 64) nt *= 2;
   const int K = sh.d_model > sh.d_ff ? sh.d_model : sh.d_ff;
   for (;;) {
-    for (int ns = kMaxStages; ns >= 4; --ns)
+    for (int ns = kMaxStages; ns >= 2; --ns) {
       if (smem_bytes(nt, ns, 2, K) <= kMaxSmemPerCta) return {nt, ns, 2};
-    for (int ns = kMaxStages; ns >= 2; --ns)
       if (smem_bytes(nt, ns, 1, K) <= kMaxSmemPerCta) return {nt, ns, 1};
+    }
     if (nt == 16) return {16, 0, 1};  // does not fit: refused by the plan
     nt /= 2;
   }

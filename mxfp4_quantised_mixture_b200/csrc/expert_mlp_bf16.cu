@@ -18,16 +18,17 @@
 //   * down: 128 rows of the [D][F] matrix; output y_perm [S][D] bf16.
 // Warp roles (4 + 4 * kDecodeGroups warps):
 //   warp 0       weight producer: the tile's E8M0 scale bytes (one bulk
-//                copy) and per stage the packed codes (TMA, 4 KB) into an
-//                8-deep ring released by the decoders
+//                copy) and per stage the packed codes (TMA, 4 KB) into a
+//                9- or 12-deep ring released by the decoders
 //   warp 1       token producer and tensor-memory owner: per stage NT token
-//                rows x 64 bf16 (TMA, 128-byte swizzle) into slot j of a ring
-//                whose slot j pairs with A slot j in tensor memory
-//   warps 2, 3   MMA issuers, taking even and odd stages into two fp32
-//                accumulators in tensor memory (D0, D1); one commit per stage
-//                frees both the token slot and the A slot.  Two issuers keep
-//                the tensor core fed: one thread issues an M=128, N<=64 MMA
-//                only every ~50 cycles and a commit costs a few hundred.
+//                rows x 64 bf16 (TMA, 128-byte swizzle) into a ring of token
+//                slots released by the MMAs
+//   warps 2, 3   MMA issuers (one or two by tile width), taking stages
+//                round-robin into one fp32 accumulator each in tensor memory
+//                (D0, D1); per stage one commit frees the token slot and one
+//                the A slot.  Two issuers keep the tensor core fed where one
+//                CTA has the SM: one thread issues an M=128, N<=64 MMA only
+//                every ~50 cycles and a commit costs a few hundred.
 //   warpgroups   decoders, taking stages round-robin: each thread owns one
 //                weight row (its tensor-memory lane), turns 64 codes per
 //                stage into exact bf16 and writes them to the stage's A slot;
@@ -55,21 +56,31 @@ namespace {
 constexpr int BK = 64;                // K elements per pipeline stage
 constexpr int BM = 128;               // weight rows per tile (MMA M)
 constexpr int W_STAGE = BM * BK / 2;  // packed code bytes per stage
-constexpr int NSW = 8;                // weight ring depth
 constexpr int kDecodeGroups = 3;
 constexpr int kDecWarp0 = 4;
 constexpr int kThreads = 32 * (kDecWarp0 + 4 * kDecodeGroups);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestWaitNs = 200000ull;  // the injected wait of test_timeout_cta
 
-// per token-tile width: token/A slots and MMA issuers (tensor memory holds
-// NMMA accumulators of NT columns plus NA A slots of 32 columns)
-__host__ __device__ constexpr int slots_for(int NT) {
-  return NT == 32 ? 6 : (NT == 64 ? 4 : (NT == 128 ? 6 : 4));
+// Per token-tile width: MMA issuers, token slots (shared memory, NT rows
+// each), A slots (tensor memory, 32 columns each) and weight-ring depth.
+// Tensor memory holds NMMA accumulators of NT columns plus the A slots;
+// narrow tiles run two CTAs per SM (256 columns each), wide ones one.
+// An mbarrier waiter names a phase by its parity alone, so it must never
+// wait on a phase two ahead of the barrier's current one (the parity would
+// match the phase before, already complete).  Every waiter below therefore
+// sees every phase of each barrier it waits on: a weight stage and an A slot
+// always go to the same decode group (NSW and NA multiples of the group
+// count) and an A slot or token slot always to the same MMA issuer (NA and
+// NX multiples of the issuer count).
+__host__ __device__ constexpr int issuers_for(int NT) { return (NT == 32 || NT == 128) ? 2 : 1; }
+__host__ __device__ constexpr int a_slots_for(int) { return 6; }
+__host__ __device__ constexpr int x_slots_for(int NT) {
+  return NT == 32 ? 6 : (NT == 64 ? 4 : (NT == 128 ? 8 : 4));
 }
-__host__ __device__ constexpr int issuers_for(int NT) { return NT <= 128 ? 2 : 1; }
+__host__ __device__ constexpr int nsw_for(int NT) { return NT <= 64 ? 9 : 12; }
 __host__ __device__ constexpr int tmem_cols_for(int NT) {
-  return issuers_for(NT) * NT + slots_for(NT) * 32 <= 256 ? 256 : 512;
+  return issuers_for(NT) * NT + a_slots_for(NT) * 32 <= 256 ? 256 : 512;
 }
 
 struct SmemLayout {
@@ -79,10 +90,10 @@ struct SmemLayout {
 __host__ __device__ inline SmemLayout smem_layout(int NT, int K) {
   SmemLayout L;
   L.x_off = 0;
-  L.w_off = L.x_off + slots_for(NT) * NT * 128;
-  L.s_off = L.w_off + NSW * W_STAGE;
+  L.w_off = L.x_off + x_slots_for(NT) * NT * 128;
+  L.s_off = L.w_off + nsw_for(NT) * W_STAGE;
   L.bar_off = L.s_off + ((BM * (K / 32) + 127) / 128) * 128;
-  L.total = L.bar_off + 512;
+  L.total = L.bar_off + 1024;
   return L;
 }
 
@@ -155,7 +166,12 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
                        const Tile* __restrict__ tiles, const int* __restrict__ n_tiles,
                        int rows_per_expert, int K, int out_ld, uint16_t* __restrict__ out,
                        int32_t* __restrict__ status, int fail_cta) {
-  constexpr int NA = slots_for(NT);
+  constexpr int NA = a_slots_for(NT);
+  constexpr int NX = x_slots_for(NT);
+  constexpr int NSW = nsw_for(NT);
+  static_assert(NSW % kDecodeGroups == 0 && NA % kDecodeGroups == 0, "slot -> decode group");
+  static_assert(NA % issuers_for(NT) == 0 && NX % issuers_for(NT) == 0, "slot -> MMA issuer");
+  static_assert(NT > 64 || tmem_cols_for(NT) == 256, "two CTAs per SM share tensor memory");
   constexpr int NMMA = issuers_for(NT);
   constexpr int X_STAGE = NT * 128;
   constexpr int TMEM_COLS = tmem_cols_for(NT);
@@ -173,10 +189,11 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* wfull = bars;              // [NSW] weight codes landed
   uint64_t* wempty = wfull + NSW;      // [NSW] weight codes read by the decoders
-  uint64_t* xfull = wempty + NSW;      // [NA]  token rows landed
-  uint64_t* afull = xfull + NA;        // [NA]  A slot written by the decoders
-  uint64_t* consumed = afull + NA;     // [NA]  MMA done with token slot + A slot
-  uint64_t* sbar = consumed + NA;      // scales landed
+  uint64_t* xfull = wempty + NSW;      // [NX]  token rows landed
+  uint64_t* xfree = xfull + NX;        // [NX]  MMAs done with the token slot
+  uint64_t* afull = xfree + NX;        // [NA]  A slot written by the decoders
+  uint64_t* afree = afull + NA;        // [NA]  MMAs done with the A slot
+  uint64_t* sbar = afree + NA;         // scales landed
   uint64_t* dfull = sbar + 1;          // accumulators complete (one commit per issuer)
   uint64_t* never = dfull + 1;         // completed by nothing (the injected test wait)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never + 1);
@@ -193,10 +210,13 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
       tc::mbar_init(&wfull[s], 1);
       tc::mbar_init(&wempty[s], 4);
     }
-    for (int j = 0; j < NA; ++j) {
+    for (int j = 0; j < NX; ++j) {
       tc::mbar_init(&xfull[j], 1);
+      tc::mbar_init(&xfree[j], 1);
+    }
+    for (int j = 0; j < NA; ++j) {
       tc::mbar_init(&afull[j], 4);
-      tc::mbar_init(&consumed[j], 1);
+      tc::mbar_init(&afree[j], 1);
     }
     tc::mbar_init(sbar, 1);
     tc::mbar_init(dfull, NMMA);
@@ -260,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
     if (lane == 0) {
       int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        const int j = kb % NA, n = kb / NA;
-        if (n > 0 && !tc::mbar_wait(&consumed[j], (n - 1) & 1, abort_flag, kWaitLimitNs)) {
+        const int j = kb % NX, n = kb / NX;
+        if (n > 0 && !tc::mbar_wait(&xfree[j], (n - 1) & 1, abort_flag, kWaitLimitNs)) {
           abort_cta(abort_flag, status);
           break;
         }
@@ -269,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
         tc::tma_load_2d(xs + j * X_STAGE, &map_x, &xfull[j], kb * BK, tile.row0);
         ++issued;
       }
-      for (int kb = max(0, issued - NA); kb < issued; ++kb)
-        tc::mbar_drain(&xfull[kb % NA], (kb / NA) & 1, kWaitLimitNs / 8);
+      for (int kb = max(0, issued - NX); kb < issued; ++kb)
+        tc::mbar_drain(&xfull[kb % NX], (kb / NX) & 1, kWaitLimitNs / 8);
     }
   } else if (warp < kDecWarp0) {
     // ---------------------------------------------------------- MMA issuers
@@ -288,20 +308,22 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
         ok = false;
       }
       for (int kb = mi; ok && kb < KB; kb += NMMA) {
-        const int j = kb % NA;
-        const uint32_t par = (kb / NA) & 1;
-        if (!tc::mbar_wait(&xfull[j], par, abort_flag, kWaitLimitNs) ||
-            !tc::mbar_wait(&afull[j], par, abort_flag, kWaitLimitNs)) {
+        const int jx = kb % NX, ja = kb % NA;
+        if (!tc::mbar_wait(&xfull[jx], (kb / NX) & 1, abort_flag, kWaitLimitNs) ||
+            !tc::mbar_wait(&afull[ja], (kb / NA) & 1, abort_flag, kWaitLimitNs)) {
           abort_cta(abort_flag, status);
           break;
         }
         tc::tc_fence_after();
-        const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(xs + j * X_STAGE));
+        const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(xs + jx * X_STAGE));
 #pragma unroll
         for (int i = 0; i < BK / 16; ++i)
-          tc::mma_bf16_ts(tmem_d, tmem_a + j * 32 + i * 8, bdesc + static_cast<uint64_t>(i * 2),
+          tc::mma_bf16_ts(tmem_d, tmem_a + ja * 32 + i * 8, bdesc + static_cast<uint64_t>(i * 2),
                           IDESC, (done | i) != 0);
-        tc::mma_commit(&consumed[j]);
+        // each commit completes once every MMA this thread issued so far has
+        // finished: the token slot and the A slot are free again
+        tc::mma_commit(&xfree[jx]);
+        tc::mma_commit(&afree[ja]);
         ++done;
       }
       // completes once every MMA this thread issued has finished (also on
@@ -333,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
     const bool row_live = GATE_UP || (mt * BM + m < rows_per_expert);
     const uint8_t* my_scales = ssm + srow_s * kscale;
     for (int kb = g; ok && kb < KB; kb += kDecodeGroups) {
-      const int s = kb % NSW, j = kb % NA;
+      const int s = kb % NSW, j = kb % NA;  // weight stage, A slot
       if (!warp_wait(&wfull[s], (kb / NSW) & 1, abort_flag)) {
         abort_cta(abort_flag, status);
         ok = false;
@@ -357,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
       decode32(p0, s0, o0);
       decode32(p1, s1, o1);
       const int use = kb / NA;
-      if (use > 0 && !warp_wait(&consumed[j], (use - 1) & 1, abort_flag)) {
+      if (use > 0 && !warp_wait(&afree[j], (use - 1) & 1, abort_flag)) {
         abort_cta(abort_flag, status);
         ok = false;
         break;

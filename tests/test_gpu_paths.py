@@ -229,3 +229,43 @@ def test_both_paths_on_one_shape(dev, T, D, F, E, k):
         assert beyond <= 0.01
         # each path may carry one flipped h against the exact result
         assert_layer_close(a, b, f"{what} paths", 2 * hflip if what == "y" else None)
+
+
+# ------------------------------------------------------ repeated calls
+
+
+@pytest.mark.parametrize("T,D,F,E,k,path", [
+    (200, 2880, 2880, 32, 4, BF),  # tiles of 64 rows (one MMA issuer, two CTAs per SM)
+    (64, 2880, 2880, 32, 4, BF),   # tiles of 32 rows (two issuers, two CTAs per SM)
+    (400, 1024, 1024, 32, 4, BF),  # tiles of 128 rows (two issuers, one CTA per SM)
+    (2000, 512, 768, 16, 4, BF),   # tiles of 256 rows
+    (64, 2880, 2880, 32, 4, BS),   # the block-scaled path at the 20B decode batch
+])
+def test_paths_repeatable(dev, T, D, F, E, k, path):
+    # Every output element is one fixed-order sum, so repeated calls agree
+    # bit for bit; outputs are prefilled with NaN so an element that no
+    # kernel wrote, or one that read a ring slot out of turn, shows up.
+    shape = moe.make_shape(T, E, k, D, F)
+    x, lg, gu, dn = _case(T, D, F, E, k, seed=11 + T)
+    host, wdev = _weights(gu, dn, dev)
+    xp, offsets, _ = _permuted(x, lg, k, E)
+    S = xp.shape[0]
+    ws = moe.alloc_workspace(shape, WS_OF[path], dev)
+    xd, od = to_dev_u16(xp, dev), torch.from_numpy(offsets).to(dev)
+    first = None
+    for rep in range(8):
+        h = torch.full((S, F), float("nan"), dtype=torch.bfloat16, device=dev)
+        y = torch.full((S, D), float("nan"), dtype=torch.bfloat16, device=dev)
+        moe.moe_expert_mlp_ex(xd, od, shape, *wdev, h, y, ws, path=path)
+        torch.cuda.synchronize()
+        assert int(ws[:4].view(torch.int32).item()) == moe.MOE_OK
+        got = (bf16_np(h), bf16_np(y))
+        if first is None:
+            first = got
+            oh, oy = oracle.expert_mlp(xp, offsets, *host)
+            assert_layer_close(got[0], oh, f"h {T},{D},{F},{E},{k}")
+            assert_layer_close(got[1], oy, f"y {T},{D},{F},{E},{k}",
+                               h_flip_bound(oh, offsets, decoded_down(host[2], host[3])))
+        else:
+            assert np.array_equal(got[0], first[0]), f"h differs on call {rep}"
+            assert np.array_equal(got[1], first[1]), f"y differs on call {rep}"
