@@ -16,19 +16,20 @@
 //     interleaved in tensor memory (lane 2j = gate j, lane 2j+1 = up j), so
 //     the SwiGLU epilogue pairs neighbouring lanes; output h [S][F] bf16.
 //   * down: 128 rows of the [D][F] matrix; output y_perm [S][D] bf16.
-// Warp roles (4 + 4 * kDecodeGroups warps):
+// Warp roles (4 + 4 * decode groups warps; 3 groups for tiles of up to 64
+// rows, which run two CTAs per SM, 4 for wider tiles):
 //   warp 0       weight producer: the tile's E8M0 scale bytes (one bulk
 //                copy) and per stage the packed codes (TMA, 4 KB) into a
-//                9- or 12-deep ring released by the decoders
+//                ring of 8 or 9 stages released by the decoders
 //   warp 1       token producer and tensor-memory owner: per stage NT token
-//                rows x 64 bf16 (TMA, 128-byte swizzle) into a ring of token
-//                slots released by the MMAs
-//   warps 2, 3   MMA issuers (one or two by tile width), taking stages
-//                round-robin into one fp32 accumulator each in tensor memory
-//                (D0, D1); per stage one commit frees the token slot and one
-//                the A slot.  Two issuers keep the tensor core fed where one
-//                CTA has the SM: one thread issues an M=128, N<=64 MMA only
-//                every ~50 cycles and a commit costs a few hundred.
+//                rows x 64 bf16 (TMA, 128-byte swizzle) into slot j of a ring
+//                whose slot j pairs with A slot j in tensor memory
+//   warps 2, 3   MMA issuers (two for tiles of 32 and 128 rows, else one),
+//                taking stages round-robin into one fp32 accumulator each in
+//                tensor memory (D0, D1); one commit per stage frees both the
+//                token slot and the A slot.  One thread issues an M=128,
+//                N<=64 MMA only every ~50 cycles and a commit costs a few
+//                hundred, so a second issuer helps where the MMAs are short.
 //   warpgroups   decoders, taking stages round-robin: each thread owns one
 //                weight row (its tensor-memory lane), turns 64 codes per
 //                stage into exact bf16 and writes them to the stage's A slot;
@@ -56,31 +57,29 @@ namespace {
 constexpr int BK = 64;                // K elements per pipeline stage
 constexpr int BM = 128;               // weight rows per tile (MMA M)
 constexpr int W_STAGE = BM * BK / 2;  // packed code bytes per stage
-constexpr int kDecodeGroups = 3;
 constexpr int kDecWarp0 = 4;
-constexpr int kThreads = 32 * (kDecWarp0 + 4 * kDecodeGroups);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestWaitNs = 200000ull;  // the injected wait of test_timeout_cta
 
-// Per token-tile width: MMA issuers, token slots (shared memory, NT rows
-// each), A slots (tensor memory, 32 columns each) and weight-ring depth.
-// Tensor memory holds NMMA accumulators of NT columns plus the A slots;
-// narrow tiles run two CTAs per SM (256 columns each), wide ones one.
+// Per token-tile width: decode groups, MMA issuers, token/A slot pairs and
+// weight-ring depth.  Tensor memory holds NMMA accumulators of NT columns
+// plus the A slots (32 columns each); narrow tiles run two CTAs per SM (256
+// columns each), wide ones one.
 // An mbarrier waiter names a phase by its parity alone, so it must never
 // wait on a phase two ahead of the barrier's current one (the parity would
 // match the phase before, already complete).  Every waiter below therefore
-// sees every phase of each barrier it waits on: a weight stage and an A slot
-// always go to the same decode group (NSW and NA multiples of the group
-// count) and an A slot or token slot always to the same MMA issuer (NA and
-// NX multiples of the issuer count).
+// sees every phase of each barrier it waits on: a weight stage and a slot
+// pair always go to the same decode group (ring depths multiples of the
+// group count) and a slot pair always to the same MMA issuer.
+__host__ __device__ constexpr int groups_for(int NT) { return NT <= 64 ? 3 : 4; }
+__host__ __device__ constexpr int threads_for(int NT) { return 32 * (kDecWarp0 + 4 * groups_for(NT)); }
 __host__ __device__ constexpr int issuers_for(int NT) { return (NT == 32 || NT == 128) ? 2 : 1; }
-__host__ __device__ constexpr int a_slots_for(int) { return 6; }
-__host__ __device__ constexpr int x_slots_for(int NT) {
-  return NT == 32 ? 6 : (NT == 64 ? 4 : (NT == 128 ? 8 : 4));
+__host__ __device__ constexpr int slots_for(int NT) {
+  return NT <= 64 ? 6 : (NT == 128 ? 8 : 4);
 }
-__host__ __device__ constexpr int nsw_for(int NT) { return NT <= 64 ? 9 : 12; }
+__host__ __device__ constexpr int nsw_for(int NT) { return NT <= 64 ? 9 : 8; }
 __host__ __device__ constexpr int tmem_cols_for(int NT) {
-  return issuers_for(NT) * NT + a_slots_for(NT) * 32 <= 256 ? 256 : 512;
+  return issuers_for(NT) * NT + slots_for(NT) * 32 <= 256 ? 256 : 512;
 }
 
 struct SmemLayout {
@@ -90,10 +89,10 @@ struct SmemLayout {
 __host__ __device__ inline SmemLayout smem_layout(int NT, int K) {
   SmemLayout L;
   L.x_off = 0;
-  L.w_off = L.x_off + x_slots_for(NT) * NT * 128;
+  L.w_off = L.x_off + slots_for(NT) * NT * 128;
   L.s_off = L.w_off + nsw_for(NT) * W_STAGE;
   L.bar_off = L.s_off + ((BM * (K / 32) + 127) / 128) * 128;
-  L.total = L.bar_off + 1024;
+  L.total = L.bar_off + 512;
   return L;
 }
 
@@ -160,19 +159,18 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 template <int NT, bool GATE_UP>
-__global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per SM for narrow tiles
+__global__ void __launch_bounds__(threads_for(NT), NT <= 64 ? 2 : 1)  // two CTAs per SM for narrow tiles
     grouped_mxfp4_gemm(const __grid_constant__ CUtensorMap map_w,
                        const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ scales,
                        const Tile* __restrict__ tiles, const int* __restrict__ n_tiles,
                        int rows_per_expert, int K, int out_ld, uint16_t* __restrict__ out,
                        int32_t* __restrict__ status, int fail_cta) {
-  constexpr int NA = a_slots_for(NT);
-  constexpr int NX = x_slots_for(NT);
-  constexpr int NSW = nsw_for(NT);
-  static_assert(NSW % kDecodeGroups == 0 && NA % kDecodeGroups == 0, "slot -> decode group");
-  static_assert(NA % issuers_for(NT) == 0 && NX % issuers_for(NT) == 0, "slot -> MMA issuer");
-  static_assert(NT > 64 || tmem_cols_for(NT) == 256, "two CTAs per SM share tensor memory");
+  constexpr int NA = slots_for(NT);
   constexpr int NMMA = issuers_for(NT);
+  constexpr int NSW = nsw_for(NT);
+  constexpr int DG = groups_for(NT);
+  static_assert(NSW % DG == 0 && NA % DG == 0 && NA % NMMA == 0, "slot owners");
+  static_assert(NT > 64 || tmem_cols_for(NT) == 256, "two CTAs per SM share tensor memory");
   constexpr int X_STAGE = NT * 128;
   constexpr int TMEM_COLS = tmem_cols_for(NT);
   constexpr uint32_t IDESC = tc::idesc_bf16_f32(BM, NT);
@@ -189,11 +187,10 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* wfull = bars;              // [NSW] weight codes landed
   uint64_t* wempty = wfull + NSW;      // [NSW] weight codes read by the decoders
-  uint64_t* xfull = wempty + NSW;      // [NX]  token rows landed
-  uint64_t* xfree = xfull + NX;        // [NX]  MMAs done with the token slot
-  uint64_t* afull = xfree + NX;        // [NA]  A slot written by the decoders
-  uint64_t* afree = afull + NA;        // [NA]  MMAs done with the A slot
-  uint64_t* sbar = afree + NA;         // scales landed
+  uint64_t* xfull = wempty + NSW;      // [NA]  token rows landed
+  uint64_t* afull = xfull + NA;        // [NA]  A slot written by the decoders
+  uint64_t* consumed = afull + NA;     // [NA]  MMA done with token slot + A slot
+  uint64_t* sbar = consumed + NA;      // scales landed
   uint64_t* dfull = sbar + 1;          // accumulators complete (one commit per issuer)
   uint64_t* never = dfull + 1;         // completed by nothing (the injected test wait)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never + 1);
@@ -210,13 +207,10 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
       tc::mbar_init(&wfull[s], 1);
       tc::mbar_init(&wempty[s], 4);
     }
-    for (int j = 0; j < NX; ++j) {
-      tc::mbar_init(&xfull[j], 1);
-      tc::mbar_init(&xfree[j], 1);
-    }
     for (int j = 0; j < NA; ++j) {
+      tc::mbar_init(&xfull[j], 1);
       tc::mbar_init(&afull[j], 4);
-      tc::mbar_init(&afree[j], 1);
+      tc::mbar_init(&consumed[j], 1);
     }
     tc::mbar_init(sbar, 1);
     tc::mbar_init(dfull, NMMA);
@@ -280,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
     if (lane == 0) {
       int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        const int j = kb % NX, n = kb / NX;
-        if (n > 0 && !tc::mbar_wait(&xfree[j], (n - 1) & 1, abort_flag, kWaitLimitNs)) {
+        const int j = kb % NA, n = kb / NA;
+        if (n > 0 && !tc::mbar_wait(&consumed[j], (n - 1) & 1, abort_flag, kWaitLimitNs)) {
           abort_cta(abort_flag, status);
           break;
         }
@@ -289,8 +283,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
         tc::tma_load_2d(xs + j * X_STAGE, &map_x, &xfull[j], kb * BK, tile.row0);
         ++issued;
       }
-      for (int kb = max(0, issued - NX); kb < issued; ++kb)
-        tc::mbar_drain(&xfull[kb % NX], (kb / NX) & 1, kWaitLimitNs / 8);
+      for (int kb = max(0, issued - NA); kb < issued; ++kb)
+        tc::mbar_drain(&xfull[kb % NA], (kb / NA) & 1, kWaitLimitNs / 8);
     }
   } else if (warp < kDecWarp0) {
     // ---------------------------------------------------------- MMA issuers
@@ -308,22 +302,20 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
         ok = false;
       }
       for (int kb = mi; ok && kb < KB; kb += NMMA) {
-        const int jx = kb % NX, ja = kb % NA;
-        if (!tc::mbar_wait(&xfull[jx], (kb / NX) & 1, abort_flag, kWaitLimitNs) ||
-            !tc::mbar_wait(&afull[ja], (kb / NA) & 1, abort_flag, kWaitLimitNs)) {
+        const int j = kb % NA;
+        const uint32_t par = (kb / NA) & 1;
+        if (!tc::mbar_wait(&xfull[j], par, abort_flag, kWaitLimitNs) ||
+            !tc::mbar_wait(&afull[j], par, abort_flag, kWaitLimitNs)) {
           abort_cta(abort_flag, status);
           break;
         }
         tc::tc_fence_after();
-        const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(xs + jx * X_STAGE));
+        const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(xs + j * X_STAGE));
 #pragma unroll
         for (int i = 0; i < BK / 16; ++i)
-          tc::mma_bf16_ts(tmem_d, tmem_a + ja * 32 + i * 8, bdesc + static_cast<uint64_t>(i * 2),
+          tc::mma_bf16_ts(tmem_d, tmem_a + j * 32 + i * 8, bdesc + static_cast<uint64_t>(i * 2),
                           IDESC, (done | i) != 0);
-        // each commit completes once every MMA this thread issued so far has
-        // finished: the token slot and the A slot are free again
-        tc::mma_commit(&xfree[jx]);
-        tc::mma_commit(&afree[ja]);
+        tc::mma_commit(&consumed[j]);
         ++done;
       }
       // completes once every MMA this thread issued has finished (also on
@@ -354,8 +346,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
     // rows past the end of the expert's matrix (last down tile) read no scales
     const bool row_live = GATE_UP || (mt * BM + m < rows_per_expert);
     const uint8_t* my_scales = ssm + srow_s * kscale;
-    for (int kb = g; ok && kb < KB; kb += kDecodeGroups) {
-      const int s = kb % NSW, j = kb % NA;  // weight stage, A slot
+    for (int kb = g; ok && kb < KB; kb += DG) {
+      const int s = kb % NSW, j = kb % NA;
       if (!warp_wait(&wfull[s], (kb / NSW) & 1, abort_flag)) {
         abort_cta(abort_flag, status);
         ok = false;
@@ -379,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
       decode32(p0, s0, o0);
       decode32(p1, s1, o1);
       const int use = kb / NA;
-      if (use > 0 && !warp_wait(&afree[j], (use - 1) & 1, abort_flag)) {
+      if (use > 0 && !warp_wait(&consumed[j], (use - 1) & 1, abort_flag)) {
         abort_cta(abort_flag, status);
         ok = false;
         break;
@@ -398,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
     if (ok) {
       tc::tc_fence_after();
       uint8_t* stg = xs;  // every token slot has been consumed: reuse as staging
-      for (int c = g * 16; c < NT; c += 16 * kDecodeGroups) {
+      for (int c = g * 16; c < NT; c += 16 * DG) {
         float v[16];
         uint32_t r[16];
         tc::tmem_ld16(tmem + lane_base + c, r);
@@ -438,10 +430,10 @@ __global__ void __launch_bounds__(kThreads, NT <= 64 ? 2 : 1)  // two CTAs per S
       }
     }
     // all decoder warps meet before the coalesced stores
-    asm volatile("bar.sync 1, %0;" ::"r"(128 * kDecodeGroups));
+    asm volatile("bar.sync 1, %0;" ::"r"(128 * DG));
     if (ok && !*abort_flag) {
       const int tid = threadIdx.x - kDecWarp0 * 32;
-      const int nthr = 128 * kDecodeGroups;
+      const int nthr = 128 * DG;
       if (GATE_UP) {
         // h rows: 64 features (128 bytes = 8 x 16 B) per token
         const int f0 = mt * 64;
@@ -562,7 +554,7 @@ moe_status launch_gemm(const CUtensorMap& mw, const CUtensorMap& mx, const uint8
                        int out_ld, uint16_t* out, int32_t* status, int fail_cta,
                        cudaStream_t stream) {
   const int smem = smem_layout(NT, K).total + 1024;
-  return launch(grouped_mxfp4_gemm<NT, GATE_UP>, dim3(grid_x, grid_y), dim3(kThreads), smem,
+  return launch(grouped_mxfp4_gemm<NT, GATE_UP>, dim3(grid_x, grid_y), dim3(threads_for(NT)), smem,
                 stream, mw, mx, scales, tiles, n_tiles, R, K, out_ld, out, status,
                 fail_cta);
 }
