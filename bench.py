@@ -71,6 +71,8 @@ UNQUANTISED_AT = "20b_decode"
 # GEMMs' tile list), the row gather (or, on the block-scaled path, the split
 # of the rows straight from x), the gate/up GEMM, the down GEMM, combine
 LAUNCHES_PER_LAYER = 6
+LAUNCH_NOTE = ("step = one replay of a CUDA graph holding one moe_layer_forward call (its six "
+               "kernels), captured once per workload; 'eager' = the same call launched per step")
 
 # dram bytes (read + write) of one moe_expert_mlp call per workload, from ncu
 # captures of the kernels whose code (comments and whitespace aside) hashes
@@ -420,6 +422,40 @@ def quantised_weights(moe, ctx, wl, keep_first_chunk=False, keep_bf16=False):
                                           "bf16": (bf_gu, bf_dn) if keep_bf16 else None}
 
 
+def captured(torch, fn):
+    """A CUDA graph of fn(stream): one call on a side stream first (so any
+    one-time set-up of the call happens outside the capture), then the
+    capture.  Replaying it launches the same kernels with the same arguments
+    on the current stream."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn(side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    return g
+
+
+def replay_ms(torch, g, flush, stream, steps: int) -> list:
+    """Per-replay device ms of graph g, L2 flushed (outside the events) before
+    each replay, two untimed replays first."""
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps + 2):
+        flush.fill_(i & 0xFF)
+        if i >= 2:
+            st[i - 2].record(stream)
+        g.replay()
+        if i >= 2:
+            en[i - 2].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in zip(st, en)]
+
+
 def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
     """Time one workload: the layer step, the expert MLP's roofline, e2e
     (with layer_only, the layer step alone)."""
@@ -437,15 +473,22 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
     out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
     ws = moe.alloc_workspace(shape, moe.WS_LAYER, dev)
 
-    def layer():
-        moe.moe_layer_forward(x, logits, shape, wgu_q, wgu_s, wdn_q, wdn_s, out, ws, stream)
+    def layer(s=stream):
+        moe.moe_layer_forward(x, logits, shape, wgu_q, wgu_s, wdn_q, wdn_s, out, ws, s)
 
+    def layer_status():
+        st = int(ws[:4].view(torch.int32).item())
+        if st != 0:
+            raise RuntimeError("layer reported device status %d" % st)
+
+    # the step as a serving loop runs it: moe_layer_forward captured once into
+    # a CUDA graph (its six kernels, no host work per step), replayed per step
+    graph = captured(torch, layer)
     for _ in range(args.warmup):
         flush.fill_(1)
-        layer()
+        graph.replay()
     torch.cuda.synchronize()
-    if int(ws[:4].view(torch.int32).item()) != 0:
-        raise RuntimeError("layer reported device status %d" % int(ws[:4].view(torch.int32).item()))
+    layer_status()
 
     # ---- timed region: K steps, events around each step, L2 flushed between
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -459,25 +502,40 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         starts[i].record(stream)
-        layer()
+        graph.replay()
         ends[i].record(stream)
     torch.cuda.synchronize()
     ctx.barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
-    if int(ws[:4].view(torch.int32).item()) != 0:
-        raise RuntimeError("layer reported device status %d" % int(ws[:4].view(torch.int32).item()))
+    layer_status()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = reduce_max(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(ctx.world, T, args.steps, total_ms)
+
+    # the same steps as eager calls (host planning and six launches per step)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e_starts[i].record(stream)
+        layer()
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    layer_status()
+    eager_ms = reduce_max(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), dev) / args.steps
+    eager = {"ms_per_step": eager_ms, "value": ctx.world * T / (eager_ms / 1e3)}
+    del graph
     if layer_only:
         return {"value": value, "ms_per_step": ms_per_step, "config": config_dict(wl),
+                "launch": LAUNCH_NOTE, "eager": eager,
                 "clocks": clk, "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
                 "step_ms_min": min(step_ms), "step_ms_max": max(step_ms)}
 
     # ---- roofline of the grouped expert MLP: the same step through the
-    #      individual calls, with events around moe_expert_mlp
+    #      individual calls: route and permute once, then moe_expert_mlp
+    #      captured into a CUDA graph and replayed between events
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     tw = torch.empty((T, k), dtype=torch.float32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
@@ -488,20 +546,14 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
     h = torch.empty((S, F), dtype=torch.bfloat16, device=dev)
     yp = torch.empty((S, D), dtype=torch.bfloat16, device=dev)
     ws_mlp = moe.alloc_workspace(shape, moe.WS_EXPERT_MLP, dev)
-    m_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    m_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for i in range(args.steps + 2):
-        flush.fill_(i & 0xFF)
-        moe.moe_route(logits, k, idx, tw, stream)
-        moe.moe_permute(idx, x, shape, counts, offsets, ss, sp, xp, None, stream)
-        if i >= 2:
-            m_starts[i - 2].record(stream)
-        moe.moe_expert_mlp(xp, offsets, shape, wgu_q, wgu_s, wdn_q, wdn_s, h, yp, ws_mlp, stream)
-        if i >= 2:
-            m_ends[i - 2].record(stream)
-        moe.moe_combine(yp, sp, tw, shape, out, stream)
-    torch.cuda.synchronize()
-    mlp_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(m_starts, m_ends))
+    moe.moe_route(logits, k, idx, tw, stream)
+    moe.moe_permute(idx, x, shape, counts, offsets, ss, sp, xp, None, stream)
+    g_mlp = captured(torch, lambda s: moe.moe_expert_mlp(xp, offsets, shape, wgu_q, wgu_s, wdn_q,
+                                                         wdn_s, h, yp, ws_mlp, s))
+    mlp_ms = statistics.mean(replay_ms(torch, g_mlp, flush, stream, args.steps))
+    del g_mlp
+    if int(ws_mlp[:4].view(torch.int32).item()) != 0:
+        raise RuntimeError("expert MLP reported device status %d" % int(ws_mlp[:4].view(torch.int32).item()))
     touched = int((counts > 0).sum().item())
     mlp_bytes = touched * expert_bytes(wl) + 2 * S * D * 2
     hbm, tc_burst, tc_sust, peak_kind = ctx.peaks
@@ -552,7 +604,7 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
 
     return {
         "value": value, "ms_per_step": ms_per_step, "config": config_dict(wl),
-        "roofline": roof,
+        "launch": LAUNCH_NOTE, "eager": eager, "roofline": roof,
         "layer_roofline": {"bytes": layer_bytes, "flops": layer_flops,
                            "frac_of_measured": t_roof_meas / (ms_per_step / 1e3),
                            "frac_of_spec_8TBs_2.25PF": t_roof_spec / (ms_per_step / 1e3),
@@ -591,25 +643,18 @@ def unquantised_timing(moe, ctx, wl, weights, bf16_weights) -> dict:
     ws_u = moe.alloc_workspace(shape, moe.WS_EXPERT_MLP_UNQUANTISED, dev)
     bf_gu, bf_dn = bf16_weights
     calls = {
-        "mxfp4": lambda: moe.moe_expert_mlp(xp, offsets, shape, *weights, h, yp, ws_q, stream),
-        "bf16": lambda: moe.moe_expert_mlp_unquantised(xp, offsets, shape, bf_gu, bf_dn, h, yp,
-                                                       ws_u, stream),
+        "mxfp4": lambda s: moe.moe_expert_mlp(xp, offsets, shape, *weights, h, yp, ws_q, s),
+        "bf16": lambda s: moe.moe_expert_mlp_unquantised(xp, offsets, shape, bf_gu, bf_dn, h, yp,
+                                                         ws_u, s),
     }
     torch.cuda.synchronize()
     touched = int((counts > 0).sum().item())
-    out = {"call": "moe_expert_mlp_unquantised vs moe_expert_mlp", "workload": wl.name}
+    out = {"call": "moe_expert_mlp_unquantised vs moe_expert_mlp (CUDA graph replays)",
+           "workload": wl.name}
     for name, call in calls.items():
-        st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-        en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-        for i in range(steps + 2):
-            flush.fill_(i & 0xFF)
-            if i >= 2:
-                st[i - 2].record(stream)
-            call()
-            if i >= 2:
-                en[i - 2].record(stream)
-        torch.cuda.synchronize()
-        ms = statistics.mean(a.elapsed_time(b) for a, b in zip(st, en))
+        g = captured(torch, call)
+        ms = statistics.mean(replay_ms(torch, g, flush, stream, steps))
+        del g
         wbytes = touched * (expert_bytes(wl) if name == "mxfp4" else 3 * D * F * 2)
         out[name] = {"ms": ms, "weight_bytes": wbytes,
                      "GB/s": (wbytes + 2 * S * D * 2) / (ms / 1e3) / 1e9}
@@ -633,19 +678,12 @@ def router_timing(moe, ctx, wl):
                                 .view(np.int16)).to(dev).view(torch.bfloat16)
     r_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     r_w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    for i in range(steps + 2):
-        flush.fill_(i & 0xFF)
-        if i >= 2:
-            st[i - 2].record(stream)
-        moe.moe_router_topk(x, w_router, k, r_idx, r_w, None, None, stream)
-        if i >= 2:
-            en[i - 2].record(stream)
-    torch.cuda.synchronize()
-    ms = statistics.mean(a.elapsed_time(b) for a, b in zip(st, en))
+    g = captured(torch, lambda s: moe.moe_router_topk(x, w_router, k, r_idx, r_w, None, None, s))
+    ms = statistics.mean(replay_ms(torch, g, flush, stream, steps))
+    del g
     nbytes = T * D * 2 + E * D * 2 + T * k * 8
-    return {"call": "moe_router_topk", "workload": wl.name, "ms": ms, "bytes": nbytes,
+    return {"call": "moe_router_topk (CUDA graph replays)", "workload": wl.name, "ms": ms,
+            "bytes": nbytes,
             "GB/s": nbytes / (ms / 1e3) / 1e9, "TFLOP/s": 2.0 * T * D * E / (ms / 1e3) / 1e12}
 
 
@@ -686,6 +724,8 @@ def run_ours(args):
         if name == UNQUANTISED_AT:
             extras["unquantised"] = unquantised_timing(moe, ctx, wl, weights, keep["bf16"])
             keep["bf16"] = None
+        if name == "20b_decode" and name != names[0]:
+            extras["router_decode"] = router_timing(moe, ctx, wl)
         if name == names[0]:
             extras["router"] = router_timing(moe, ctx, wl)
             extras["quantize"] = quantiser_timings(moe, keep["first"], ctx.flush, ctx.stream,
@@ -708,7 +748,9 @@ def run_ours(args):
         "gpu_launches": head["gpu_launches"],
         "wall_s_timed_region": head["wall_s_timed_region"],
         "step_ms_min": head["step_ms_min"], "step_ms_max": head["step_ms_max"],
-        "router": extras.get("router"), "quantize": extras.get("quantize"),
+        "launch": head["launch"], "eager": head["eager"],
+        "router": extras.get("router"), "router_decode": extras.get("router_decode"),
+        "quantize": extras.get("quantize"),
         "unquantised": extras.get("unquantised"),
         "per_workload": {n: r for n, r in results.items() if n != names[0]},
     }

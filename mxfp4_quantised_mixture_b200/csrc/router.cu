@@ -181,25 +181,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         tv[j] = -INFINITY;
         ti[j] = 0x7FFFFFFF;
       }
-      for (int e = 0; e < E; ++e) {
-        const float* pe = part + e * MT + m;
-        float v = tc::ld_cluster_f32(tc::cluster_addr(pe, 0));
-        for (int r = 1; r < cs; ++r) v += tc::ld_cluster_f32(tc::cluster_addr(pe, r));
-        if (logits) logits[static_cast<int64_t>(t) * E + e] = v;
-        // experts arrive in index order: an equal value never displaces an
-        // earlier one, so ties keep the lower index
-        if (better(v, e, tv[7], ti[7])) {
-          tv[7] = v;
-          ti[7] = e;
+      // the partials of rank r sit at base[r] + 4 (e MT + m) in the cluster
+      // window; the loads of four experts x all ranks are issued before any
+      // is added, so their latencies overlap
+      uint32_t base[8];
 #pragma unroll
-          for (int j = 7; j > 0; --j) {
-            if (better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
-              const float fv = tv[j];
-              tv[j] = tv[j - 1];
-              tv[j - 1] = fv;
-              const int fi = ti[j];
-              ti[j] = ti[j - 1];
-              ti[j - 1] = fi;
+      for (int r = 0; r < 8; ++r) base[r] = r < cs ? tc::cluster_addr(part + m, r) : 0u;
+      for (int e0 = 0; e0 < E; e0 += 4) {
+        float pv[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+            pv[u][r] = (r < cs && e0 + u < E)
+                           ? tc::ld_cluster_f32(base[r] + static_cast<uint32_t>((e0 + u) * MT * 4))
+                           : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u;
+          if (e >= E) break;
+          float v = pv[u][0];
+#pragma unroll
+          for (int r = 1; r < 8; ++r)
+            if (r < cs) v += pv[u][r];
+          if (logits) logits[static_cast<int64_t>(t) * E + e] = v;
+          // experts arrive in index order: an equal value never displaces an
+          // earlier one, so ties keep the lower index
+          if (better(v, e, tv[7], ti[7])) {
+            tv[7] = v;
+            ti[7] = e;
+#pragma unroll
+            for (int j = 7; j > 0; --j) {
+              if (better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
+                const float fv = tv[j];
+                tv[j] = tv[j - 1];
+                tv[j - 1] = fv;
+                const int fi = ti[j];
+                ti[j] = ti[j - 1];
+                ti[j - 1] = fi;
+              }
             }
           }
         }
