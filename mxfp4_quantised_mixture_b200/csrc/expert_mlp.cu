@@ -89,8 +89,13 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (6 + kEpiWarps);
 constexpr int kMaxStages = 12;      // copy ring depth limit (stage slot s also owns scale slot s)
 constexpr int kSlotCols = 8 * WPS;  // per stage and window: 4 token-scale + 4 weight-scale columns
-constexpr int kAccCols = 128;       // tensor-memory columns per accumulator (N <= 128)
-constexpr int kTmemCols = 512;      // two accumulators, then the scale slots
+// Tensor memory: two accumulators, then the scale slots.  One CTA per SM
+// holds all 512 columns (accumulators 128 apart); with two CTAs per SM
+// (16-token tiles) each holds 128: accumulators of 2 NT = 32 columns and up
+// to 4 stage slots.
+__host__ __device__ constexpr int acc_cols_for(bool two) { return two ? 32 : 128; }
+__host__ __device__ constexpr int tmem_cols_for(bool two) { return two ? 128 : 512; }
+constexpr int kTwoMaxStages = (128 - 2 * 32) / (8 * 2);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestWaitNs = 200000ull;  // the injected wait of test_timeout_cta
 
@@ -207,15 +212,18 @@ struct GemmArgs {
   int fail_cta;
 };
 
-template <int NT, bool GATE_UP>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int NT, bool GATE_UP, bool TWO>
+__global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
     grouped_mx_gemm(const __grid_constant__ CUtensorMap map_w,
                     const __grid_constant__ CUtensorMap map_w_tail,
                     const __grid_constant__ CUtensorMap map_x, const GemmArgs args) {
   constexpr int XR = 2 * NT;  // token piece rows per window
   constexpr uint32_t X_BYTES = XR * BKS;
   constexpr uint32_t IDESC = tc::idesc_mx(tc::kFmtE2M1, tc::kFmtE4M3, BN, XR);
+  constexpr int kAccCols = acc_cols_for(TWO);
+  constexpr int kTmemCols = tmem_cols_for(TWO);
   static_assert(XR >= 16 && XR <= kAccCols && (X_BYTES % 1024) == 0, "token tile of 8..64 tokens");
+  static_assert(!TWO || NT == 16, "two CTAs per SM only for 16-token tiles");
   const int rows_per_expert = args.rows_per_expert, K = args.K, NS = args.NS, NB = args.NB;
   const Tile* __restrict__ tiles = args.tiles;
   int32_t* status = args.status;
@@ -758,28 +766,40 @@ bool make_piece_map(CUtensorMap* map, const uint8_t* pieces, int64_t padded_rows
 }
 
 struct GemmConfig {
-  int NT, NS, NB;
+  int NT, NS, NB, CPS;
 };
 
 constexpr int kMaxSmemPerCta = 227 * 1024;
+// two CTAs share an SM's 228 KB, each with 1 KB reserved
+constexpr int kTwoSmemPerCta = 112 * 1024;
 
 int smem_bytes(int NT, int NS, int NB, int K) { return smem_layout(NT, NS, NB, K).total + 1024; }
 
-// token-tile width: about twice the mean rows per expert, 16..64; then the
-// deepest copy ring (up to 12 stages), its weight-scale block double-buffered
-// when that costs no stage
+// token-tile width: about twice the mean rows per expert, 16..64.  16-token
+// tiles run two CTAs per SM when two stages fit in half the shared memory:
+// one thread issuing every copy of an SM's ring was measured to cap the
+// stream of the 4-bit weight boxes well below the HBM rate, and two CTAs
+// (two issuing threads, two rings) lift it.  Otherwise one CTA per SM with
+// the deepest copy ring (up to 12 stages), its weight-scale block
+// double-buffered when that costs no stage.
 GemmConfig choose_config(const moe_shape& sh) {
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
   const int64_t want = 2 * ((S + sh.E - 1) / sh.E);
   int nt = 16;
   while (nt < want && nt < 64) nt *= 2;
   const int K = sh.d_model > sh.d_ff ? sh.d_model : sh.d_ff;
+  if (nt == 16) {
+    for (int ns = kTwoMaxStages; ns >= 2; --ns) {
+      if (smem_bytes(16, ns, 2, K) <= kTwoSmemPerCta) return {16, ns, 2, 2};
+      if (smem_bytes(16, ns, 1, K) <= kTwoSmemPerCta) return {16, ns, 1, 2};
+    }
+  }
   for (;;) {
     for (int ns = kMaxStages; ns >= 2; --ns) {
-      if (smem_bytes(nt, ns, 2, K) <= kMaxSmemPerCta) return {nt, ns, 2};
-      if (smem_bytes(nt, ns, 1, K) <= kMaxSmemPerCta) return {nt, ns, 1};
+      if (smem_bytes(nt, ns, 2, K) <= kMaxSmemPerCta) return {nt, ns, 2, 1};
+      if (smem_bytes(nt, ns, 1, K) <= kMaxSmemPerCta) return {nt, ns, 1, 1};
     }
-    if (nt == 16) return {16, 0, 1};  // does not fit: refused by the plan
+    if (nt == 16) return {16, 0, 1, 1};  // does not fit: refused by the plan
     nt /= 2;
   }
 }
@@ -803,34 +823,37 @@ bool allow_smem(Kern kern, std::atomic<uint64_t>& done) {
   return true;
 }
 
-template <int NT, bool GATE_UP>
+template <int NT, bool GATE_UP, bool TWO>
 bool prepare_gemm() {
   static std::atomic<uint64_t> done{0};
-  return allow_smem(grouped_mx_gemm<NT, GATE_UP>, done);
+  return allow_smem(grouped_mx_gemm<NT, GATE_UP, TWO>, done);
 }
 
-bool prepare_nt(int NT) {
+bool prepare_nt(int NT, int CPS) {
   switch (NT) {
     case 16:
-      return prepare_gemm<16, true>() && prepare_gemm<16, false>();
+      return CPS == 2 ? prepare_gemm<16, true, true>() && prepare_gemm<16, false, true>()
+                      : prepare_gemm<16, true, false>() && prepare_gemm<16, false, false>();
     case 32:
-      return prepare_gemm<32, true>() && prepare_gemm<32, false>();
+      return prepare_gemm<32, true, false>() && prepare_gemm<32, false, false>();
     default:
-      return prepare_gemm<64, true>() && prepare_gemm<64, false>();
+      return prepare_gemm<64, true, false>() && prepare_gemm<64, false, false>();
   }
 }
 
-template <int NT, bool GATE_UP>
+template <int NT, bool GATE_UP, bool TWO>
 moe_status launch_gemm(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& mwt,
                        const CUtensorMap& mx, const GemmArgs& a, int max_items,
                        cudaStream_t stream) {
   const int smem = smem_bytes(NT, P.NS, P.NB, a.K);
-  const int grid = max_items < sm_count() ? max_items : sm_count();
-  // each CTA holds all 512 tensor-memory columns: ask for enough shared
-  // memory that no second CTA shares the SM
-  const int smem_launch = smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
-  return launch(grouped_mx_gemm<NT, GATE_UP>, dim3(grid), dim3(kThreads), smem_launch, stream,
-                mw, mwt, mx, a);
+  const int slots = (TWO ? 2 : 1) * sm_count();
+  const int grid = max_items < slots ? max_items : slots;
+  // one CTA per SM holds all 512 tensor-memory columns: it asks for enough
+  // shared memory that no second CTA shares the SM
+  const int smem_launch =
+      TWO || smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
+  return launch(grouped_mx_gemm<NT, GATE_UP, TWO>, dim3(grid), dim3(kThreads), smem_launch,
+                stream, mw, mwt, mx, a);
 }
 
 template <bool GATE_UP>
@@ -838,11 +861,12 @@ moe_status launch_nt(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& 
                      const CUtensorMap& mx, const GemmArgs& a, int max_items, cudaStream_t st) {
   switch (P.NT) {
     case 16:
-      return launch_gemm<16, GATE_UP>(P, mw, mwt, mx, a, max_items, st);
+      return P.CPS == 2 ? launch_gemm<16, GATE_UP, true>(P, mw, mwt, mx, a, max_items, st)
+                        : launch_gemm<16, GATE_UP, false>(P, mw, mwt, mx, a, max_items, st);
     case 32:
-      return launch_gemm<32, GATE_UP>(P, mw, mwt, mx, a, max_items, st);
+      return launch_gemm<32, GATE_UP, false>(P, mw, mwt, mx, a, max_items, st);
     default:
-      return launch_gemm<64, GATE_UP>(P, mw, mwt, mx, a, max_items, st);
+      return launch_gemm<64, GATE_UP, false>(P, mw, mwt, mx, a, max_items, st);
   }
 }
 
@@ -889,6 +913,7 @@ moe_status mx_plan(MlpPlan* p, void* ws) {
   P.NT = cfg.NT;
   P.NS = cfg.NS;
   P.NB = cfg.NB;
+  P.CPS = cfg.CPS;
   P.max_tiles = W.max_tiles;
   P.padded_rows = W.padded_rows;
   p->n_tiles = reinterpret_cast<int*>(base + W.n_tiles);
@@ -903,7 +928,7 @@ moe_status mx_plan(MlpPlan* p, void* ws) {
       !make_piece_map(&P.m_x, P.pieces_x, W.padded_rows, D, cfg.NT) ||
       !make_piece_map(&P.m_h, P.pieces_h, W.padded_rows, F, cfg.NT))
     return MOE_ERR_CUDA;
-  if (!prepare_nt(cfg.NT)) return MOE_ERR_CUDA;
+  if (!prepare_nt(cfg.NT, cfg.CPS)) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -47,6 +47,7 @@ size_t bf_workspace(const moe_shape& sh);
 struct MxPlan {
   CUtensorMap m_gu, m_gu_t, m_dn, m_dn_t, m_x, m_h;
   int NT, NS, NB;
+  int CPS;  // CTAs per SM of the GEMMs (1, or 2 for 16-token tiles)
   int64_t max_tiles, padded_rows;
   uint8_t *pieces_x, *pieces_h;
   uint32_t *words_x, *words_h;
