@@ -173,7 +173,6 @@ __global__ void __launch_bounds__(threads_for(NT), NT <= 64 ? 2 : 1)  // two CTA
   static_assert(NT > 64 || tmem_cols_for(NT) == 256, "two CTAs per SM share tensor memory");
   constexpr int X_STAGE = NT * 128;
   constexpr int TMEM_COLS = tmem_cols_for(NT);
-  constexpr uint32_t IDESC = tc::idesc_bf16_f32(BM, NT);
   // a CTA beyond the tile count leaves before any set-up
   if (static_cast<int>(blockIdx.y) >= __ldg(n_tiles)) return;
 
@@ -198,6 +197,11 @@ __global__ void __launch_bounds__(threads_for(NT), NT <= 64 ? 2 : 1)  // two CTA
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Tile tile = tiles[blockIdx.y];
+  // the MMAs cover the tile's rows rounded up to 16, not the whole width: a
+  // ragged tile (an expert's last, or a cold expert's only) costs the tensor
+  // core only its own rows
+  const int NV = min(NT, (tile.nrows + 15) & ~15);
+  const uint32_t IDESC = tc::idesc_bf16_f32(BM, NV);
   const int mt = blockIdx.x;
   const int KB = K / BK;
   const int kscale = K / 32;
@@ -390,7 +394,7 @@ __global__ void __launch_bounds__(threads_for(NT), NT <= 64 ? 2 : 1)  // two CTA
     if (ok) {
       tc::tc_fence_after();
       uint8_t* stg = xs;  // every token slot has been consumed: reuse as staging
-      for (int c = g * 16; c < NT; c += 16 * DG) {
+      for (int c = g * 16; c < NV; c += 16 * DG) {
         float v[16];
         uint32_t r[16];
         tc::tmem_ld16(tmem + lane_base + c, r);

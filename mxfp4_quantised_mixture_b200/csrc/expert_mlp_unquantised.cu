@@ -70,7 +70,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        uint16_t* __restrict__ out, int32_t* __restrict__ status) {
   constexpr int NS = stages_for(NT);
   constexpr int STAGE = stage_bytes(NT);
-  constexpr uint32_t IDESC = tc::idesc_bf16_f32(BM, NT);
   constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
   if (static_cast<int>(blockIdx.y) >= __ldg(n_tiles)) return;  // whole CTA, before any set-up
 
@@ -86,6 +85,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Tile tile = tiles[blockIdx.y];
+  // the MMAs cover the tile's rows rounded up to 16, not the whole width: a
+  // ragged tile (an expert's last, or a cold expert's only) costs the tensor
+  // core only its own rows
+  const int NV = min(NT, (tile.nrows + 15) & ~15);
+  const uint32_t IDESC = tc::idesc_bf16_f32(BM, NV);
   const int mt = blockIdx.x;
   const int KB = K / BK;
 
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t* stg = reinterpret_cast<uint16_t*>(smem);
     if (ok) {
       tc::tc_fence_after();
-      for (int c = 0; c < NT; c += 16) {
+      for (int c = 0; c < NV; c += 16) {
         uint32_t r[16];
         tc::tmem_ld16(tmem + lane_base + c, r);
         tc::tmem_ld_wait();

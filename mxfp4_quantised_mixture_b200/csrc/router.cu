@@ -7,9 +7,9 @@
 // The router scores every token against every expert; the routing that
 // follows is the one moe_route computes from given logits.
 //
-// One cluster of up to 8 CTAs per 128 tokens, each CTA taking a contiguous
-// share of the reduction axis (so a decode batch of a few tokens still
-// spreads over several SMs).  The scores are a bf16 GEMM on the tensor core:
+// Batches of T * E <= 16384 take a small kernel on the CUDA cores, one CTA
+// per token (below).  Larger ones: one cluster of up to 8 CTAs per 128
+// tokens, each CTA taking a contiguous share of the reduction axis.  The scores are a bf16 GEMM on the tensor core:
 // tokens on the MMA's M side (128), the experts on N (E padded to a multiple
 // of 16, at most 256), K = D in stages of 64 (one 128-byte swizzle row of
 // bf16), both operands by TMA into shared memory, the fp32 accumulator in
@@ -39,6 +39,7 @@ constexpr int MT = 128;                 // tokens per CTA (MMA M)
 constexpr int A_BYTES = MT * BKR * 2;   // token rows per stage
 constexpr int NSR = 4;                  // stages in the ring
 constexpr int kThreads = 192;
+constexpr int64_t kSmallRouterWork = 16384;  // T * E at or below which the small-batch kernel runs
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __host__ __device__ inline int smem_bytes_router(int npad) {
@@ -47,6 +48,138 @@ __host__ __device__ inline int smem_bytes_router(int npad) {
 
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
+}
+
+// Running top-8 list (value descending, index ascending).  Experts arrive in
+// index order, so an equal value never displaces an earlier one and ties keep
+// the lower index.
+__device__ __forceinline__ void insert_top8(float v, int e, float (&tv)[8], int (&ti)[8]) {
+  if (better(v, e, tv[7], ti[7])) {
+    tv[7] = v;
+    ti[7] = e;
+#pragma unroll
+    for (int j = 7; j > 0; --j) {
+      if (better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
+        const float fv = tv[j];
+        tv[j] = tv[j - 1];
+        tv[j - 1] = fv;
+        const int fi = ti[j];
+        ti[j] = ti[j - 1];
+        ti[j - 1] = fi;
+      }
+    }
+  }
+}
+
+// Softmax over the first k of the list, summed in the order of moe_route's
+// butterfly over lanes j = 0..7 (zero beyond k), and the stores of token t.
+__device__ __forceinline__ void store_topk(const float (&tv)[8], const int (&ti)[8], int k,
+                                           int64_t t, int32_t* __restrict__ idx,
+                                           float* __restrict__ wts) {
+  float ex[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) ex[j] = j < k ? expf(tv[j] - tv[0]) : 0.f;
+  const float z = ((ex[0] + ex[4]) + (ex[2] + ex[6])) + ((ex[1] + ex[5]) + (ex[3] + ex[7]));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k) {
+      idx[t * k + j] = ti[j];
+      wts[t * k + j] = ex[j] / z;
+    }
+  }
+}
+
+// Small batches (a few tokens against the experts): one CTA per token, no
+// tensor core.  The token's row is staged in shared memory; warp w scores
+// experts w, w + warps, ...: lane l takes the 16-byte vectors l, l + 32, ...
+// of the row in order and the warp adds its lanes with a butterfly, a fixed
+// order.  Warp 0 then picks the top 8 by rounds of a warp arg-max over the
+// experts not yet taken (value descending, index ascending: the order of the
+// running list) and stores the routing.  The router matrix is read once per token,
+// from L2 after the first.
+constexpr int kSmallThreads = 512;
+
+__global__ void __launch_bounds__(kSmallThreads)
+    router_small_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, int D,
+                        int E, int k, float* __restrict__ logits, int32_t* __restrict__ idx,
+                        float* __restrict__ wts) {
+  extern __shared__ __align__(16) uint8_t small_smem[];
+  uint4* xs = reinterpret_cast<uint4*>(small_smem);                 // [D / 8]
+  float* sc = reinterpret_cast<float*>(small_smem + D * 2);         // [E]
+  const int64_t t = blockIdx.x;
+  const int nv = D / 8;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + t * D);
+  for (int j = threadIdx.x; j < nv; j += blockDim.x) xs[j] = __ldg(xr + j);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  // two experts per pass, so a lane has both rows' loads in flight
+  for (int e0 = warp; e0 < E; e0 += 2 * nw) {
+    const int e1 = e0 + nw;
+    const uint4* w0 = reinterpret_cast<const uint4*>(w + static_cast<int64_t>(e0) * D);
+    const uint4* w1 = e1 < E ? reinterpret_cast<const uint4*>(w + static_cast<int64_t>(e1) * D) : w0;
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 6
+    for (int j = lane; j < nv; j += 32) {
+      const uint4 a = xs[j];
+      const uint4 b0 = __ldg(w0 + j);
+      const uint4 b1 = __ldg(w1 + j);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bv0[4] = {b0.x, b0.y, b0.z, b0.w}, bv1[4] = {b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float xl = __uint_as_float(av[h] << 16), xh = __uint_as_float(av[h] & 0xFFFF0000u);
+        acc0 = fmaf(xl, __uint_as_float(bv0[h] << 16), acc0);
+        acc0 = fmaf(xh, __uint_as_float(bv0[h] & 0xFFFF0000u), acc0);
+        acc1 = fmaf(xl, __uint_as_float(bv1[h] << 16), acc1);
+        acc1 = fmaf(xh, __uint_as_float(bv1[h] & 0xFFFF0000u), acc1);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      acc0 += __shfl_xor_sync(0xFFFFFFFFu, acc0, o);
+      acc1 += __shfl_xor_sync(0xFFFFFFFFu, acc1, o);
+    }
+    if (lane == 0) {
+      sc[e0] = acc0;
+      if (e1 < E) sc[e1] = acc1;
+    }
+  }
+  __syncthreads();
+  if (logits)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) logits[t * E + e] = sc[e];
+  if (warp == 0) {
+    // the top 8 in the order of the running list (value descending, index
+    // ascending): 8 rounds of a warp arg-max over the experts not yet taken
+    float tv[8];
+    int ti[8];
+    uint32_t taken = 0;  // bit c: expert 32 c + lane is already in the list (E <= 256)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7FFFFFFF;
+      // lane l owns experts l, l + 32, ...
+      for (int c = 0; 32 * c + lane < E; ++c) {
+        const int e = 32 * c + lane;
+        if (!((taken >> c) & 1u) && better(sc[e], e, bv, bi)) {
+          bv = sc[e];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      tv[r] = bv;
+      ti[r] = bi;
+      if (bi != 0x7FFFFFFF && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    }
+    if (lane == 0) store_topk(tv, ti, k, t, idx, wts);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -206,38 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int r = 1; r < 8; ++r)
             if (r < cs) v += pv[u][r];
           if (logits) logits[static_cast<int64_t>(t) * E + e] = v;
-          // experts arrive in index order: an equal value never displaces an
-          // earlier one, so ties keep the lower index
-          if (better(v, e, tv[7], ti[7])) {
-            tv[7] = v;
-            ti[7] = e;
-#pragma unroll
-            for (int j = 7; j > 0; --j) {
-              if (better(tv[j], ti[j], tv[j - 1], ti[j - 1])) {
-                const float fv = tv[j];
-                tv[j] = tv[j - 1];
-                tv[j - 1] = fv;
-                const int fi = ti[j];
-                ti[j] = ti[j - 1];
-                ti[j - 1] = fi;
-              }
-            }
-          }
+          insert_top8(v, e, tv, ti);
         }
       }
-      // softmax over the first k, summed in the order of moe_route's
-      // butterfly over lanes j = 0..7 (zero beyond k)
-      float ex[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) ex[j] = j < k ? expf(tv[j] - tv[0]) : 0.f;
-      const float z = ((ex[0] + ex[4]) + (ex[2] + ex[6])) + ((ex[1] + ex[5]) + (ex[3] + ex[7]));
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < k) {
-          idx[static_cast<int64_t>(t) * k + j] = ti[j];
-          wts[static_cast<int64_t>(t) * k + j] = ex[j] / z;
-        }
-      }
+      store_topk(tv, ti, k, t, idx, wts);
     }
   }
 
@@ -290,6 +395,31 @@ moe_status router_launch(const uint16_t* x, const uint16_t* w_router, int T, int
                          float* logits, int32_t* idx, float* wts, int32_t* status,
                          cudaStream_t stream) {
   if (T == 0) return MOE_OK;
+  if (static_cast<int64_t>(T) * E <= kSmallRouterWork) {
+    // a few tokens: one CTA per token on the CUDA cores (a tensor-core tile
+    // of 128 tokens would be mostly padding, and its reduction over a
+    // cluster costs more than the scores)
+    const int smem = D * 2 + E * 4;
+    if (smem > 48 * 1024) {
+      static std::atomic<uint64_t> small_done{0};
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+      if (!bit || !(small_done.load() & bit)) {
+        if (cudaFuncSetAttribute(router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 16384 * 2 + 256 * 4) != cudaSuccess) {
+          cudaGetLastError();
+          return MOE_ERR_CUDA;
+        }
+        small_done.fetch_or(bit);
+      }
+    }
+    return launch(router_small_kernel, dim3(T), dim3(kSmallThreads), smem, stream, x, w_router,
+                  D, E, k, logits, idx, wts);
+  }
   const int npad = (E + 15) / 16 * 16;
   CUtensorMap mx, mw;
   if (!make_rows_map(&mx, x, T, D, MT) || !make_rows_map(&mw, w_router, E, D, npad))

@@ -54,16 +54,21 @@ def _check(x_np, w_np, k, dev):
     assert np.array_equal(idx, idx2) and np.array_equal(tw.view(np.uint32), tw2.view(np.uint32))
 
 
+# T * E <= 16384 runs the small-batch kernel (one CTA per token), larger
+# batches the tensor-core kernel; both kinds of shape are here
 @pytest.mark.parametrize("T,D,E,k", [(64, 2880, 32, 4), (128, 2880, 128, 4), (1, 64, 8, 4),
-                                     (200, 256, 33, 2), (300, 512, 256, 8), (17, 192, 16, 1)])
+                                     (200, 256, 33, 2), (17, 192, 16, 1), (1, 16384, 256, 8),
+                                     (300, 512, 256, 8), (600, 512, 32, 4), (1000, 128, 64, 8),
+                                     (2048, 2880, 128, 4)])
 def test_router_topk(cuda_device, T, D, E, k):
     x = syn.normal_bf16(30, 910 + E, (T, D))
     w = syn.normal_bf16(30, 911 + E, (E, D), sigma=1.0 / np.sqrt(D))
     _check(x, w, k, cuda_device)
 
 
-def test_router_ties_go_to_the_lower_index(cuda_device):
-    T, D, E, k = 130, 128, 24, 4
+@pytest.mark.parametrize("T", [130, 1000])
+def test_router_ties_go_to_the_lower_index(cuda_device, T):
+    D, E, k = 128, 24, 4
     x = syn.normal_bf16(31, 920, (T, D))
     w = syn.normal_bf16(31, 921, (E, D), sigma=0.1)
     w[5] = w[2]    # experts 2 and 5 always score the same
