@@ -77,8 +77,13 @@ LAUNCH_NOTE = ("step = one replay of a CUDA graph holding one moe_layer_forward 
 # dram bytes (read + write) of one moe_expert_mlp call per workload, from ncu
 # captures of the kernels whose code (comments and whitespace aside) hashes
 # to TRAFFIC_SRC_SHA; reported only while that code is unchanged
-TRAFFIC_BYTES: dict[str, int] = {}
-TRAFFIC_SRC_SHA = ""
+TRAFFIC_BYTES: dict[str, int] = {
+    # gate/up + down GEMM dram__bytes_read.sum + dram__bytes_write.sum, one
+    # launch each, from `ncu --set full` captures of the layer-only benchmark
+    "120b_skewed_prefill": 615593216 + 380497664 + 496604672 + 374051072,
+    "120b_decode": 1069808000 + 6475264 + 540402000 + 6319104,
+}
+TRAFFIC_SRC_SHA = "3309b7b24f31244a"
 
 
 def parse():
