@@ -216,7 +216,9 @@ template <int NT, bool GATE_UP, bool TWO>
 __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
     grouped_mx_gemm(const __grid_constant__ CUtensorMap map_w,
                     const __grid_constant__ CUtensorMap map_w_tail,
-                    const __grid_constant__ CUtensorMap map_x, const GemmArgs args) {
+                    const __grid_constant__ CUtensorMap map_w2,
+                    const __grid_constant__ CUtensorMap map_x,
+                    const __grid_constant__ CUtensorMap map_x2, const GemmArgs args) {
   constexpr int XR = 2 * NT;  // token piece rows per window
   constexpr uint32_t X_BYTES = XR * BKS;
   constexpr uint32_t IDESC = tc::idesc_mx(tc::kFmtE2M1, tc::kFmtE4M3, BN, XR);
@@ -276,7 +278,9 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
     tc::fence_mbar_init();
     tc::tma_prefetch_desc(&map_w);
     tc::tma_prefetch_desc(&map_w_tail);
+    tc::tma_prefetch_desc(&map_w2);
     tc::tma_prefetch_desc(&map_x);
+    tc::tma_prefetch_desc(&map_x2);
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_holder, kTmemCols);
@@ -331,7 +335,17 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
           const int w0 = st * WPS;
           const int nv = min(WPS, nwin - w0);
           tc::mbar_arrive_expect_tx(&full[s_slot], nv * (W_TX + X_BYTES));
-          for (int v = 0; v < nv; ++v) {
+          if (nv == 2 && w0 + 1 < K / BKS) {
+            // two whole windows: one copy of each operand for the stage (the
+            // copy engine's cost is mostly per copy, not per byte)
+            uint8_t* wdst = wsm + s_slot * WPS * W_SMEM;
+            if (GATE_UP) {
+              tc::tma_load_5d(wdst, &map_w2, &full[s_slot], 0, 0, wrow, w0, tile.e);
+            } else {
+              tc::tma_load_4d(wdst, &map_w2, &full[s_slot], 0, wrow, w0, tile.e);
+            }
+            tc::tma_load_3d(xs + s_slot * WPS * X_BYTES, &map_x2, &full[s_slot], 0, t * XR, w0);
+          } else for (int v = 0; v < nv; ++v) {
             const int w = w0 + v;
             const int k0 = stage_k0(w, K);
             uint8_t* wdst = wsm + (s_slot * WPS + v) * W_SMEM;
@@ -726,12 +740,27 @@ bool encode(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* ba
 // (R = 2F): the box takes a gate row and its up row for 64 consecutive f,
 // interleaved; down: 128 consecutive rows.  `main` walks the windows at
 // multiples of 128 codes, `tail` is the single window [K - 128, K).
-bool make_weight_maps(CUtensorMap* main, CUtensorMap* tail, const uint8_t* q, int E, int R,
-                      int K, bool gate_up) {
+bool make_weight_maps(CUtensorMap* main, CUtensorMap* tail, CUtensorMap* main2, const uint8_t* q,
+                      int E, int R, int K, bool gate_up) {
   const cuuint64_t row = static_cast<cuuint64_t>(K / 2);
   const cuuint64_t mat = static_cast<cuuint64_t>(R) * row;
   const CUtensorMapDataType T = CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
   const uint8_t* tail_base = q + (K - BKS) / 2;
+  // two consecutive whole windows in one box: the window is the outer box
+  // dimension, so each lands as its own [128 rows][128 B] block
+  const cuuint64_t nwf = static_cast<cuuint64_t>(K / BKS);
+  if (gate_up) {
+    const cuuint64_t F2 = static_cast<cuuint64_t>(R / 2);
+    const cuuint64_t d2[5] = {BKS, 2, F2, nwf, static_cast<cuuint64_t>(E)};
+    const cuuint64_t s2[4] = {F2 * row, row, BKS / 2, mat};
+    const cuuint32_t b2[5] = {BKS, 2, BN / 2, 2, 1};
+    if (!encode(main2, T, 5, q, d2, s2, b2)) return false;
+  } else {
+    const cuuint64_t d2[4] = {BKS, static_cast<cuuint64_t>(R), nwf, static_cast<cuuint64_t>(E)};
+    const cuuint64_t s2[3] = {row, BKS / 2, mat};
+    const cuuint32_t b2[4] = {BKS, BN, 2, 1};
+    if (!encode(main2, T, 4, q, d2, s2, b2)) return false;
+  }
   if (gate_up) {
     const cuuint64_t F = static_cast<cuuint64_t>(R / 2);
     const cuuint64_t d5[5] = {BKS, static_cast<cuuint64_t>(K / BKS), 2, F,
@@ -757,12 +786,19 @@ bool make_weight_maps(CUtensorMap* main, CUtensorMap* tail, const uint8_t* q, in
                       : encode(tail, T, 3, tail_base, d3, s3, b3);
 }
 
-// token piece rows [2 * padded rows][K] bytes, box = 128 K x 2 NT rows
-bool make_piece_map(CUtensorMap* map, const uint8_t* pieces, int64_t padded_rows, int K, int NT) {
+// token piece rows [2 * padded rows][K] bytes, box = 128 K x 2 NT rows; the
+// second map takes two consecutive whole windows per box
+bool make_piece_map(CUtensorMap* map, CUtensorMap* map2, const uint8_t* pieces,
+                    int64_t padded_rows, int K, int NT) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(2 * padded_rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
   const cuuint32_t box[2] = {BKS, static_cast<cuuint32_t>(2 * NT)};
-  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, pieces, dims, strides, box);
+  if (!encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, pieces, dims, strides, box)) return false;
+  const cuuint64_t d2[3] = {BKS, static_cast<cuuint64_t>(2 * padded_rows),
+                            static_cast<cuuint64_t>(K / BKS)};
+  const cuuint64_t s2[2] = {static_cast<cuuint64_t>(K), BKS};
+  const cuuint32_t b2[3] = {BKS, static_cast<cuuint32_t>(2 * NT), 2};
+  return encode(map2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, pieces, d2, s2, b2);
 }
 
 struct GemmConfig {
@@ -843,7 +879,8 @@ bool prepare_nt(int NT, int CPS) {
 
 template <int NT, bool GATE_UP, bool TWO>
 moe_status launch_gemm(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& mwt,
-                       const CUtensorMap& mx, const GemmArgs& a, int max_items,
+                       const CUtensorMap& mw2, const CUtensorMap& mx, const CUtensorMap& mx2,
+                       const GemmArgs& a, int max_items,
                        cudaStream_t stream) {
   const int smem = smem_bytes(NT, P.NS, P.NB, a.K);
   const int slots = (TWO ? 2 : 1) * sm_count();
@@ -853,20 +890,21 @@ moe_status launch_gemm(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap
   const int smem_launch =
       TWO || smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
   return launch(grouped_mx_gemm<NT, GATE_UP, TWO>, dim3(grid), dim3(kThreads), smem_launch,
-                stream, mw, mwt, mx, a);
+                stream, mw, mwt, mw2, mx, mx2, a);
 }
 
 template <bool GATE_UP>
 moe_status launch_nt(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& mwt,
-                     const CUtensorMap& mx, const GemmArgs& a, int max_items, cudaStream_t st) {
+                     const CUtensorMap& mw2, const CUtensorMap& mx, const CUtensorMap& mx2,
+                     const GemmArgs& a, int max_items, cudaStream_t st) {
   switch (P.NT) {
     case 16:
-      return P.CPS == 2 ? launch_gemm<16, GATE_UP, true>(P, mw, mwt, mx, a, max_items, st)
-                        : launch_gemm<16, GATE_UP, false>(P, mw, mwt, mx, a, max_items, st);
+      return P.CPS == 2 ? launch_gemm<16, GATE_UP, true>(P, mw, mwt, mw2, mx, mx2, a, max_items, st)
+                        : launch_gemm<16, GATE_UP, false>(P, mw, mwt, mw2, mx, mx2, a, max_items, st);
     case 32:
-      return launch_gemm<32, GATE_UP, false>(P, mw, mwt, mx, a, max_items, st);
+      return launch_gemm<32, GATE_UP, false>(P, mw, mwt, mw2, mx, mx2, a, max_items, st);
     default:
-      return launch_gemm<64, GATE_UP, false>(P, mw, mwt, mx, a, max_items, st);
+      return launch_gemm<64, GATE_UP, false>(P, mw, mwt, mw2, mx, mx2, a, max_items, st);
   }
 }
 
@@ -923,10 +961,10 @@ moe_status mx_plan(MlpPlan* p, void* ws) {
   P.pieces_h = reinterpret_cast<uint8_t*>(base + W.pieces_h);
   P.words_h = reinterpret_cast<uint32_t*>(base + W.words_h);
   const int D = sh.d_model, F = sh.d_ff, E = sh.E;
-  if (!make_weight_maps(&P.m_gu, &P.m_gu_t, p->wgu_q, E, 2 * F, D, true) ||
-      !make_weight_maps(&P.m_dn, &P.m_dn_t, p->wdn_q, E, D, F, false) ||
-      !make_piece_map(&P.m_x, P.pieces_x, W.padded_rows, D, cfg.NT) ||
-      !make_piece_map(&P.m_h, P.pieces_h, W.padded_rows, F, cfg.NT))
+  if (!make_weight_maps(&P.m_gu, &P.m_gu_t, &P.m_gu2, p->wgu_q, E, 2 * F, D, true) ||
+      !make_weight_maps(&P.m_dn, &P.m_dn_t, &P.m_dn2, p->wdn_q, E, D, F, false) ||
+      !make_piece_map(&P.m_x, &P.m_x2, P.pieces_x, W.padded_rows, D, cfg.NT) ||
+      !make_piece_map(&P.m_h, &P.m_h2, P.pieces_h, W.padded_rows, F, cfg.NT))
     return MOE_ERR_CUDA;
   if (!prepare_nt(cfg.NT, cfg.CPS)) return MOE_ERR_CUDA;
   return MOE_OK;
@@ -972,7 +1010,7 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
   a.pieces_out = P.pieces_h;
   a.words_out = P.words_h;
   a.fail_cta = fail_cta;
-  if ((st = launch_nt<true>(P, P.m_gu, P.m_gu_t, P.m_x, a, max_tiles * mt_gu, stream)) != MOE_OK)
+  if ((st = launch_nt<true>(P, P.m_gu, P.m_gu_t, P.m_gu2, P.m_x, P.m_x2, a, max_tiles * mt_gu, stream)) != MOE_OK)
     return st;
   // down
   a.sfx_words = P.words_h;
@@ -984,7 +1022,7 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
   a.pieces_out = nullptr;
   a.words_out = nullptr;
   a.fail_cta = -1;
-  return launch_nt<false>(P, P.m_dn, P.m_dn_t, P.m_h, a, max_tiles * mt_dn, stream);
+  return launch_nt<false>(P, P.m_dn, P.m_dn_t, P.m_dn2, P.m_h, P.m_h2, a, max_tiles * mt_dn, stream);
 }
 
 }  // namespace moe

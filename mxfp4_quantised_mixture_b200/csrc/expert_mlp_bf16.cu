@@ -260,9 +260,8 @@ __global__ void __launch_bounds__(threads_for(NT), NT <= 64 ? 2 : 1)  // two CTA
         tc::mbar_arrive_expect_tx(&wfull[s], W_STAGE);
         uint8_t* wdst = wsm + s * W_STAGE;
         if (GATE_UP) {
-          const int F = rows_per_expert / 2;
-          tc::tma_load_3d(wdst, &map_w, &wfull[s], kb * (BK / 2), r0, tile.e);
-          tc::tma_load_3d(wdst + W_STAGE / 2, &map_w, &wfull[s], kb * (BK / 2), F + r0, tile.e);
+          // the gate rows and the matching up rows in one copy (gate block first)
+          tc::tma_load_4d(wdst, &map_w, &wfull[s], kb * (BK / 2), r0, 0, tile.e);
         } else {
           tc::tma_load_3d(wdst, &map_w, &wfull[s], kb * (BK / 2), r0, tile.e);
         }
@@ -476,16 +475,26 @@ __global__ void __launch_bounds__(threads_for(NT), NT <= 64 ? 2 : 1)  // two CTA
 
 // ------------------------------------------------------------ host helpers
 
-// packed codes [E][R][K/2] bytes, box = (BK/2 bytes, box_rows rows, 1 expert)
-bool make_weight_map(CUtensorMap* map, const uint8_t* q, int E, int R, int K, int box_rows) {
+// packed codes [E][R][K/2] bytes.  Down: box = (BK/2 bytes, 128 rows, 1
+// expert).  Gate/up (R = 2F): box = (BK/2 bytes, 64 rows, gate and up half,
+// 1 expert), landing as 64 gate rows then the matching 64 up rows.
+bool make_weight_map(CUtensorMap* map, const uint8_t* q, int E, int R, int K, bool gate_up) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(R),
-                              static_cast<cuuint64_t>(E)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2),
-                                 static_cast<cuuint64_t>(R) * (K / 2)};
-  const cuuint32_t box[3] = {BK / 2, static_cast<cuuint32_t>(box_rows), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint64_t row = static_cast<cuuint64_t>(K / 2);
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (gate_up) {
+    const cuuint64_t F = static_cast<cuuint64_t>(R / 2);
+    const cuuint64_t dims[4] = {row, F, 2, static_cast<cuuint64_t>(E)};
+    const cuuint64_t strides[3] = {row, F * row, static_cast<cuuint64_t>(R) * row};
+    const cuuint32_t box[4] = {BK / 2, 64, 2, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(q), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  const cuuint64_t dims[3] = {row, static_cast<cuuint64_t>(R), static_cast<cuuint64_t>(E)};
+  const cuuint64_t strides[2] = {row, static_cast<cuuint64_t>(R) * row};
+  const cuuint32_t box[3] = {BK / 2, static_cast<cuuint32_t>(BM), 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(q), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -619,9 +628,9 @@ moe_status bf_plan(MlpPlan* p, void* ws) {
   p->tiles = reinterpret_cast<Tile*>(base + W.tiles);
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
   const int D = sh.d_model, F = sh.d_ff, E = sh.E;
-  if (!make_weight_map(&P.m_gu, p->wgu_q, E, 2 * F, D, 64) ||
+  if (!make_weight_map(&P.m_gu, p->wgu_q, E, 2 * F, D, true) ||
       !make_token_map(&P.m_x, p->x_perm, S, D, NT) ||
-      !make_weight_map(&P.m_dn, p->wdn_q, E, D, F, BM) || !make_token_map(&P.m_h, p->h, S, F, NT))
+      !make_weight_map(&P.m_dn, p->wdn_q, E, D, F, false) || !make_token_map(&P.m_h, p->h, S, F, NT))
     return MOE_ERR_CUDA;
   if (!prepare_nt(NT)) return MOE_ERR_CUDA;
   return MOE_OK;

@@ -46,6 +46,8 @@ size_t bf_workspace(const moe_shape& sh);
 // Block-scaled path (csrc/expert_mlp.cu)
 struct MxPlan {
   CUtensorMap m_gu, m_gu_t, m_dn, m_dn_t, m_x, m_h;
+  // the same, two 128-K windows per copy (one instruction per stage)
+  CUtensorMap m_gu2, m_dn2, m_x2, m_h2;
   int NT, NS, NB;
   int CPS;  // CTAs per SM of the GEMMs (1, or 2 for 16-token tiles)
   int64_t max_tiles, padded_rows;
