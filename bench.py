@@ -80,10 +80,11 @@ LAUNCH_NOTE = ("step = one replay of a CUDA graph holding one moe_layer_forward 
 TRAFFIC_BYTES: dict[str, int] = {
     # gate/up + down GEMM dram__bytes_read.sum + dram__bytes_write.sum, one
     # launch each, from `ncu --set full` captures of the layer-only benchmark
-    "120b_skewed_prefill": 615593216 + 380497664 + 496604672 + 374051072,
-    "120b_decode": 1069808000 + 6475264 + 540402000 + 6319104,
+    "120b_skewed_prefill": 615571200 + 381615104 + 496563968 + 374050048,
+    "120b_decode": 1069433000 + 6321920 + 540359000 + 5853952,
+    "20b_decode": 285221888 + 4876288 + 144217600 + 5410304,
 }
-TRAFFIC_SRC_SHA = "3309b7b24f31244a"
+TRAFFIC_SRC_SHA = "ebb83c9753e0c13e"
 
 
 def parse():
