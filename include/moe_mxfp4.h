@@ -189,8 +189,8 @@ MOE_API moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t 
  * aitrends.kr talk summary (4 active experts).
  * logits[t][e] = sum_d x[t][d] * w_router[e][d]: bf16 inputs, exact
  * products, fp32 accumulation in a fixed but unspecified order (on the
- * tensor core when T * E > 16384, else on the CUDA cores, one CTA per
- * token); then topk_idx / topk_w exactly as moe_route computes them from
+ * tensor core when T * E > 16384, else on the CUDA cores, one or two CTAs
+ * per token); then topk_idx / topk_w exactly as moe_route computes them from
  * those logits.
  *   x        in   [T][D] bf16, D a multiple of 64 in [64, 16384]
  *   w_router in   [E][D] bf16 (one row per expert), E <= 256

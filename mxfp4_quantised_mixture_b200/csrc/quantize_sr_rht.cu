@@ -57,36 +57,38 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
-// E2M1 magnitude code of v = |y| / scale >= 0, from v's fp64 bit fields:
-//   v >= 1:       binade e = 0, 1, 2 holds 2^e, 1.5 2^e: base code 2 + 2e + (top
-//                 mantissa bit), the other 51 mantissa bits are the fraction of
-//                 the gap (2^(e-1)) to the next code; v >= 8 saturates to 7;
-//   v in [.5, 1): base 1 (0.5), the 52 mantissa bits are the fraction of 0.5;
-//   v < .5:       base 0, fraction 2 v.
+constexpr double kTwo52 = 4503599627370496.0;  // 2^52: adding it leaves an integer in the low word
+constexpr double kTwo36 = 68719476736.0;       // 2^36: the low word then counts steps of 2^-16
+
+// E2M1 magnitude code of v = |y| / scale >= 0 (exact), without branches.
+// The code grid {0, .5, 1, 1.5, 2, 3, 4, 6} has step g = 0.5 below 2 and
+// g = 2^(e-1) in the binade [2^e, 2^(e+1)), e >= 1.  With e = max(floor(log2
+// v), 0) (from the high word of max(v, 1)), a = v / g is exact and lies in
+// [0, 2) below 1 and in [2, 4) above; the grid point below v is then n =
+// floor(a) steps, and the code is 2 e + n, plus one when rounded up, capped
+// at 7 (6.0; only a scale clamped at 254 reaches it).  Code parity equals n's
+// parity, so ties to even on the integer grid of a are ties to an even code.
+//   nearest:    adding 2^52 in round-to-nearest-even leaves n + up in the low word;
+//   stochastic: adding it rounding toward zero leaves n; up when
+//               n + u / 2^16 < a, i.e. u / 2^16 < (v - lo) / (hi - lo), with
+//               n + u / 2^16 built exactly as 2^36 + (n 2^16 + u) 2^-16 - 2^36.
+// rw holds the element's uniform in its low (half 0) or high (half 1) 16 bits.
 template <bool SR>
-__device__ __forceinline__ uint32_t e2m1_code(double v, uint32_t u) {
-  const uint32_t vh = static_cast<uint32_t>(__double2hiint(v));
-  const uint32_t vl = static_cast<uint32_t>(__double2loint(v));
-  const int ev = static_cast<int>(vh >> 20);  // v >= 0: no sign bit
-  uint32_t code;
-  if (ev >= 1023) {
-    const uint32_t base = 2u + 2u * static_cast<uint32_t>(ev - 1023) + ((vh >> 19) & 1u);
-    const uint64_t R = (static_cast<uint64_t>(vh & 0x7FFFFu) << 32) | vl;  // 51 bits
-    bool up;
-    if (SR)
-      up = (static_cast<uint64_t>(u) << 35) < R;
-    else
-      up = R > (1ull << 50) || (R == (1ull << 50) && (base & 1u));
-    code = min(base + (up ? 1u : 0u), 7u);
-  } else if (ev == 1022) {
-    const uint64_t R = (static_cast<uint64_t>(vh & 0xFFFFFu) << 32) | vl;  // 52 bits
-    const bool up = SR ? (static_cast<uint64_t>(u) << 36) < R : R >= (1ull << 51);
-    code = up ? 2u : 1u;
+__device__ __forceinline__ uint32_t e2m1_code(double v, uint32_t rw, int half) {
+  const int th = max(__double2hiint(v), 0x3FF00000);                         // max(v, 1)
+  const double inv_g = __hiloint2double(0x7FF00000 - (th & 0x7FF00000), 0);  // 2^(1 - e)
+  const double a = v * inv_g;
+  uint32_t c;
+  if (SR) {
+    const uint32_t n = static_cast<uint32_t>(__double2loint(__dadd_rz(a, kTwo52)));
+    const uint32_t lo = __byte_perm(rw, n, half ? 0x5432 : 0x5410);  // n 2^16 + u
+    const double nu = __hiloint2double(0x42300000, static_cast<int>(lo)) - kTwo36;
+    c = n + (nu < a ? 1u : 0u);
   } else {
-    const bool up = SR ? static_cast<double>(u) < v * 131072.0 : v > 0.25;
-    code = up ? 1u : 0u;
+    c = static_cast<uint32_t>(__double2loint(__dadd_rn(a, kTwo52)));
   }
-  return code;
+  c += 2u * static_cast<uint32_t>((th >> 20) - 1023);
+  return min(c, 7u);
 }
 
 template <bool RHT, bool SR>
@@ -149,26 +151,26 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
       }
     }
 
-    // block maximum of |y| through the high words (magnitude order), then
-    // the significand test of the stochastic-rounding scale rule
-    uint32_t amax_hi = 0;
+    // block maximum of |y| (exact), and the non-finite test: with the
+    // transform y[0] is the signed sum of the whole block, so any Inf or NaN
+    // input leaves it non-finite; without it, the plain sum of the block
+    double amax = 0.0, total = 0.0;
 #pragma unroll
-    for (int t = 0; t < 32; ++t)
-      amax_hi = max(amax_hi, static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu);
-    const bool nonfinite = amax_hi >= 0x7FF00000u;  // an Inf or NaN reached y
+    for (int t = 0; t < 32; ++t) {
+      amax = fmax(amax, fabs(y[t]));
+      if (!RHT) total += y[t];
+    }
+    if (RHT) total = y[0];
+    const bool nonfinite = (static_cast<uint32_t>(__double2hiint(total)) & 0x7FF00000u) == 0x7FF00000u;
+    const uint32_t amax_hi = static_cast<uint32_t>(__double2hiint(amax));
     int sb = 0;
     if (amax_hi != 0) {
+      // floor(log2 amax) - 2 + 127; with stochastic rounding one more when
+      // the significand of amax is above 1.5
       sb = static_cast<int>(amax_hi >> 20) - 1023 + 125;
       if (SR) {
         const uint32_t frac_hi = amax_hi & 0xFFFFFu;
-        bool above = frac_hi > 0x80000u;
-        if (frac_hi == 0x80000u) {  // significand 1.5 in the high word: the low words decide
-#pragma unroll
-          for (int t = 0; t < 32; ++t)
-            above |= (static_cast<uint32_t>(__double2hiint(y[t])) & 0x7FFFFFFFu) == amax_hi &&
-                     __double2loint(y[t]) != 0;
-        }
-        sb += above ? 1 : 0;
+        sb += (frac_hi > 0x80000u || (frac_hi == 0x80000u && __double2loint(amax) != 0)) ? 1 : 0;
       }
       sb = min(max(sb, 0), 254);
     }
@@ -189,12 +191,13 @@ __global__ void __launch_bounds__(kThreads) quantize_sr_rht_kernel(
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int t = 8 * g + e;
-        const uint32_t u = (rw[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-        uint32_t c = e2m1_code<SR>(fabs(y[t]) * inv_scale, u);
+        uint32_t c = e2m1_code<SR>(fabs(y[t]) * inv_scale, rw[e >> 1], e & 1);
         // sign bit: that of x without the transform (-0 included); with it,
-        // y < 0 only (a high word above 0x80000000 is a negative nonzero)
-        const uint32_t hy = static_cast<uint32_t>(__double2hiint(y[t]));
-        c |= (RHT ? (hy > 0x80000000u ? 1u : 0u) : (hy >> 31)) << 3;
+        // y < 0 only (an exact zero is +0)
+        if (RHT)
+          c |= y[t] < 0.0 ? 8u : 0u;
+        else
+          c |= (static_cast<uint32_t>(__double2hiint(y[t])) >> 28) & 8u;
         o |= c << (4 * e);
       }
       out[g] = o;

@@ -7,8 +7,8 @@
 // The router scores every token against every expert; the routing that
 // follows is the one moe_route computes from given logits.
 //
-// Batches of T * E <= 16384 take a small kernel on the CUDA cores, one CTA
-// per token (below).  Larger ones: one cluster of up to 8 CTAs per 128
+// Batches of T * E <= 16384 take a small kernel on the CUDA cores, one or
+// two CTAs per token (below).  Larger ones: one cluster of up to 8 CTAs per 128
 // tokens, each CTA taking a contiguous share of the reduction axis.  The scores are a bf16 GEMM on the tensor core:
 // tokens on the MMA's M side (128), the experts on N (E padded to a multiple
 // of 16, at most 256), K = D in stages of 64 (one 128-byte swizzle row of
@@ -89,72 +89,148 @@ __device__ __forceinline__ void store_topk(const float (&tv)[8], const int (&ti)
   }
 }
 
-// Small batches (a few tokens against the experts): one CTA per token, no
-// tensor core.  The token's row is staged in shared memory; warp w scores
-// experts w, w + warps, ...: lane l takes the 16-byte vectors l, l + 32, ...
-// of the row in order and the warp adds its lanes with a butterfly, a fixed
-// order.  Warp 0 then picks the top 8 by rounds of a warp arg-max over the
-// experts not yet taken (value descending, index ascending: the order of the
-// running list) and stores the routing.  The router matrix is read once per token,
-// from L2 after the first.
+// Small batches (a few tokens against the experts): no tensor core.  A token
+// takes a cluster of cs = 1 or 2 CTAs (2 while the batch leaves SMs idle), CTA
+// r scoring experts [r Eh, (r + 1) Eh), Eh = ceil(E / cs).  The token's row is
+// copied into shared memory asynchronously while every lane requests its share
+// of the router rows: warp w scores ROWS experts per pass (w, w + warps, ...
+// of the CTA's range), lane l takes the 16-byte vectors l, l + 32, ... of a
+// row in order, up to 12 of them per row in flight at once, and the warp adds
+// its lanes with a butterfly, a fixed order.  Every CTA writes its scores to
+// the logits and into the shared memory of the cluster's first CTA, where,
+// after a cluster barrier, warp 0 picks the top k by rounds of a warp arg-max
+// over the experts not yet taken (value descending, index ascending: the
+// order of the running list) and stores the routing.
 constexpr int kSmallThreads = 512;
+constexpr int kSmallUnroll = 12;
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
+               : "memory");
+}
+
+template <int ROWS>
+__device__ __forceinline__ void load_router_chunk(const uint4* const (&wr)[ROWS], int j0, int nv,
+                                                  uint4 (&b)[ROWS][kSmallUnroll]) {
+#pragma unroll
+  for (int i = 0; i < kSmallUnroll; ++i) {
+    const int j = j0 + 32 * i;
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) b[r][i] = j < nv ? __ldg(wr[r] + j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <int ROWS>
+__device__ __forceinline__ void dot_router_chunk(const uint4* xs, int j0, int nv,
+                                                 const uint4 (&b)[ROWS][kSmallUnroll],
+                                                 float (&acc)[ROWS]) {
+#pragma unroll
+  for (int i = 0; i < kSmallUnroll; ++i) {
+    const int j = j0 + 32 * i;
+    if (j < nv) {
+      const uint4 a = xs[j];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        const uint32_t bv[4] = {b[r][i].x, b[r][i].y, b[r][i].z, b[r][i].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          acc[r] = fmaf(__uint_as_float(av[h] << 16), __uint_as_float(bv[h] << 16), acc[r]);
+          acc[r] = fmaf(__uint_as_float(av[h] & 0xFFFF0000u), __uint_as_float(bv[h] & 0xFFFF0000u),
+                        acc[r]);
+        }
+      }
+    }
+  }
+}
+
+template <int ROWS>
 __global__ void __launch_bounds__(kSmallThreads)
     router_small_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, int D,
-                        int E, int k, float* __restrict__ logits, int32_t* __restrict__ idx,
-                        float* __restrict__ wts) {
+                        int E, int k, int cs, float* __restrict__ logits,
+                        int32_t* __restrict__ idx, float* __restrict__ wts) {
   extern __shared__ __align__(16) uint8_t small_smem[];
-  uint4* xs = reinterpret_cast<uint4*>(small_smem);                 // [D / 8]
-  float* sc = reinterpret_cast<float*>(small_smem + D * 2);         // [E]
-  const int64_t t = blockIdx.x;
+  uint4* xs = reinterpret_cast<uint4*>(small_smem);          // [D / 8]
+  float* sc = reinterpret_cast<float*>(small_smem + D * 2);  // [E], used in rank 0
+  const int rank = cs > 1 ? static_cast<int>(tc::cluster_rank()) : 0;
+  if (cs > 1) tc::cluster_arrive_relaxed();
+  const int64_t t = blockIdx.x / cs;
+  const int Eh = (E + cs - 1) / cs;
+  const int e_lo = rank * Eh, e_hi = min(E, e_lo + Eh);
   const int nv = D / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + t * D);
-  for (int j = threadIdx.x; j < nv; j += blockDim.x) xs[j] = __ldg(xr + j);
-  __syncthreads();
+  for (int j = threadIdx.x; j < nv; j += blockDim.x) cp_async16(xs + j, xr + j);
+  asm volatile("cp.async.commit_group;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  // two experts per pass, so a lane has both rows' loads in flight
-  for (int e0 = warp; e0 < E; e0 += 2 * nw) {
-    const int e1 = e0 + nw;
-    const uint4* w0 = reinterpret_cast<const uint4*>(w + static_cast<int64_t>(e0) * D);
-    const uint4* w1 = e1 < E ? reinterpret_cast<const uint4*>(w + static_cast<int64_t>(e1) * D) : w0;
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 6
-    for (int j = lane; j < nv; j += 32) {
-      const uint4 a = xs[j];
-      const uint4 b0 = __ldg(w0 + j);
-      const uint4 b1 = __ldg(w1 + j);
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-      const uint32_t bv0[4] = {b0.x, b0.y, b0.z, b0.w}, bv1[4] = {b1.x, b1.y, b1.z, b1.w};
+  const uint4* wv = reinterpret_cast<const uint4*>(w);
+  const uint4* wr[ROWS];
+  uint4 b[ROWS][kSmallUnroll];
+  int e0 = e_lo + warp;
+  // the first chunk of the first pass goes out with the token row
+  bool loaded = e0 < e_hi;
+  if (loaded) {
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float xl = __uint_as_float(av[h] << 16), xh = __uint_as_float(av[h] & 0xFFFF0000u);
-        acc0 = fmaf(xl, __uint_as_float(bv0[h] << 16), acc0);
-        acc0 = fmaf(xh, __uint_as_float(bv0[h] & 0xFFFF0000u), acc0);
-        acc1 = fmaf(xl, __uint_as_float(bv1[h] << 16), acc1);
-        acc1 = fmaf(xh, __uint_as_float(bv1[h] & 0xFFFF0000u), acc1);
-      }
+    for (int r = 0; r < ROWS; ++r) {
+      const int e = e0 + r * nw;
+      wr[r] = wv + static_cast<int64_t>(e < e_hi ? e : e0) * nv;
+    }
+    load_router_chunk<ROWS>(wr, lane, nv, b);
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  if (cs > 1) tc::cluster_wait();  // every CTA of the cluster has started
+  for (; e0 < e_hi; e0 += ROWS * nw) {
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      const int e = e0 + r * nw;
+      wr[r] = wv + static_cast<int64_t>(e < e_hi ? e : e0) * nv;
+    }
+    float acc[ROWS];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) acc[r] = 0.f;
+    for (int j0 = lane; j0 < nv; j0 += 32 * kSmallUnroll) {
+      if (!loaded) load_router_chunk<ROWS>(wr, j0, nv, b);
+      loaded = false;
+      dot_router_chunk<ROWS>(xs, j0, nv, b, acc);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      acc0 += __shfl_xor_sync(0xFFFFFFFFu, acc0, o);
-      acc1 += __shfl_xor_sync(0xFFFFFFFFu, acc1, o);
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) acc[r] += __shfl_xor_sync(0xFFFFFFFFu, acc[r], o);
     }
     if (lane == 0) {
-      sc[e0] = acc0;
-      if (e1 < E) sc[e1] = acc1;
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        const int e = e0 + r * nw;
+        if (e < e_hi) {
+          if (logits) logits[t * E + e] = acc[r];
+          if (rank == 0)
+            sc[e] = acc[r];
+          else
+            tc::st_cluster_f32(tc::cluster_addr(sc + e, 0), acc[r]);
+        }
+      }
     }
   }
-  __syncthreads();
-  if (logits)
-    for (int e = threadIdx.x; e < E; e += blockDim.x) logits[t * E + e] = sc[e];
+  if (cs > 1)
+    tc::cluster_sync();  // the other CTA's scores are in sc; it may now exit
+  else
+    __syncthreads();
+  if (rank != 0) return;
   if (warp == 0) {
-    // the top 8 in the order of the running list (value descending, index
-    // ascending): 8 rounds of a warp arg-max over the experts not yet taken
+    // the top k in the order of the running list (value descending, index
+    // ascending): k rounds of a warp arg-max over the experts not yet taken
     float tv[8];
     int ti[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      tv[r] = -INFINITY;
+      ti[r] = 0x7FFFFFFF;
+    }
     uint32_t taken = 0;  // bit c: expert 32 c + lane is already in the list (E <= 256)
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
+      if (r >= k) break;
       float bv = -INFINITY;
       int bi = 0x7FFFFFFF;
       // lane l owns experts l, l + 32, ...
@@ -399,6 +475,12 @@ moe_status router_launch(const uint16_t* x, const uint16_t* w_router, int T, int
     // a few tokens: one CTA per token on the CUDA cores (a tensor-core tile
     // of 128 tokens would be mostly padding, and its reduction over a
     // cluster costs more than the scores)
+    // two CTAs per token while the batch leaves half the SMs idle; each then
+    // requests only its half of the router matrix
+    const int cs = (E >= 2 && 2 * static_cast<int64_t>(T) <= sm_count()) ? 2 : 1;
+    const int eh = (E + cs - 1) / cs;
+    const bool two_rows = eh > kSmallThreads / 32;
+    auto kern = two_rows ? router_small_kernel<2> : router_small_kernel<1>;
     const int smem = D * 2 + E * 4;
     if (smem > 48 * 1024) {
       static std::atomic<uint64_t> small_done{0};
@@ -409,16 +491,33 @@ moe_status router_launch(const uint16_t* x, const uint16_t* w_router, int T, int
       }
       const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
       if (!bit || !(small_done.load() & bit)) {
-        if (cudaFuncSetAttribute(router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 16384 * 2 + 256 * 4) != cudaSuccess) {
-          cudaGetLastError();
-          return MOE_ERR_CUDA;
+        for (auto kf : {router_small_kernel<1>, router_small_kernel<2>}) {
+          if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   16384 * 2 + 256 * 4) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+          }
         }
         small_done.fetch_or(bit);
       }
     }
-    return launch(router_small_kernel, dim3(T), dim3(kSmallThreads), smem, stream, x, w_router,
-                  D, E, k, logits, idx, wts);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(T) * cs, 1, 1);
+    cfg.blockDim = dim3(kSmallThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = cs > 1 ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, x, w_router, D, E, k, cs, logits, idx, wts) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    return launch_status();
   }
   const int npad = (E + 15) / 16 * 16;
   CUtensorMap mx, mw;

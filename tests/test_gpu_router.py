@@ -54,9 +54,11 @@ def _check(x_np, w_np, k, dev):
     assert np.array_equal(idx, idx2) and np.array_equal(tw.view(np.uint32), tw2.view(np.uint32))
 
 
-# T * E <= 16384 runs the small-batch kernel (one CTA per token), larger
-# batches the tensor-core kernel; both kinds of shape are here
+# T * E <= 16384 runs the small-batch kernel (a cluster of two CTAs per token
+# while 2 T fits the SMs, one CTA per token above; one or two router rows per
+# warp and pass), larger batches the tensor-core kernel; all kinds are here
 @pytest.mark.parametrize("T,D,E,k", [(64, 2880, 32, 4), (128, 2880, 128, 4), (1, 64, 8, 4),
+                                     (40, 320, 65, 3), (74, 2880, 32, 4), (75, 2880, 32, 4),
                                      (200, 256, 33, 2), (17, 192, 16, 1), (1, 16384, 256, 8),
                                      (300, 512, 256, 8), (600, 512, 32, 4), (1000, 128, 64, 8),
                                      (2048, 2880, 128, 4)])
@@ -66,7 +68,7 @@ def test_router_topk(cuda_device, T, D, E, k):
     _check(x, w, k, cuda_device)
 
 
-@pytest.mark.parametrize("T", [130, 1000])
+@pytest.mark.parametrize("T", [50, 130, 1000])
 def test_router_ties_go_to_the_lower_index(cuda_device, T):
     D, E, k = 128, 24, 4
     x = syn.normal_bf16(31, 920, (T, D))
