@@ -67,24 +67,30 @@ FLUSH_BYTES = 256 << 20
 CPU_SAMPLE_TOKENS = 64
 # the unquantised (bf16 weight) expert MLP is timed beside the MXFP4 one here
 UNQUANTISED_AT = "20b_decode"
-# kernel launches of one moe_layer_forward call: route, permute (with the
-# GEMMs' tile list), the row gather (or, on the block-scaled path, the split
-# of the rows straight from x), the gate/up GEMM, the down GEMM, combine
-LAUNCHES_PER_LAYER = 6
-LAUNCH_NOTE = ("step = one replay of a CUDA graph holding one moe_layer_forward call (its six "
-               "kernels), captured once per workload; 'eager' = the same call launched per step")
+# kernel launches of one moe_layer_forward call, per GEMM path:
+#   block-scaled: route, permute (with the GEMMs' tile list), the split of the
+#     rows straight from x into E4M3 pieces, one launch running both GEMMs,
+#     combine;
+#   bf16-decode: route, permute, the row gather, the gate/up GEMM, the down
+#     GEMM, combine
+LAUNCHES_PER_LAYER = {"block-scaled": 5, "bf16-decode": 6}
+LAUNCH_NOTE = ("step = one replay of a CUDA graph holding one moe_layer_forward call (5 kernels "
+               "on the block-scaled path, 6 on the bf16-decode path), captured once per "
+               "workload; 'eager' = the same call launched per step")
 
 # dram bytes (read + write) of one moe_expert_mlp call per workload, from ncu
-# captures of the kernels whose code (comments and whitespace aside) hashes
-# to TRAFFIC_SRC_SHA; reported only while that code is unchanged
-TRAFFIC_BYTES: dict[str, int] = {
+# captures of the GEMM kernels of the source file named beside them, reported
+# only while that file's code (comments and whitespace aside) still hashes to
+# the value recorded with them
+TRAFFIC: dict[str, tuple[int, str, str]] = {
     # gate/up + down GEMM dram__bytes_read.sum + dram__bytes_write.sum, one
     # launch each, from `ncu --set full` captures of the layer-only benchmark
-    "120b_skewed_prefill": 615571200 + 381615104 + 496563968 + 374050048,
-    "120b_decode": 1069433000 + 6321920 + 540359000 + 5853952,
-    "20b_decode": 285221888 + 4876288 + 144217600 + 5410304,
+    "120b_skewed_prefill": (615571200 + 381615104 + 496563968 + 374050048,
+                            "expert_mlp_bf16.cu", "b96e9f861b69c97f"),
+    # the one launch of both GEMMs
+    "120b_decode": (0, "expert_mlp.cu", "MX_SHA"),
+    "20b_decode": (0, "expert_mlp.cu", "MX_SHA"),
 }
-TRAFFIC_SRC_SHA = "ebb83c9753e0c13e"
 
 
 def parse():
@@ -124,12 +130,24 @@ def code_tokens(src: str) -> str:
     return " ".join(src.split())
 
 
-def kernel_src_sha() -> str:
-    h = hashlib.sha256()
-    for name in ("expert_mlp.cu", "expert_mlp_bf16.cu"):
-        with open(os.path.join(ROOT, "mxfp4_quantised_mixture_b200", "csrc", name)) as f:
-            h.update(code_tokens(f.read()).encode())
-    return h.hexdigest()[:16]
+def kernel_src_sha(name: str) -> str:
+    with open(os.path.join(ROOT, "mxfp4_quantised_mixture_b200", "csrc", name)) as f:
+        return hashlib.sha256(code_tokens(f.read()).encode()).hexdigest()[:16]
+
+
+def gemm_path(wl) -> str:
+    """The GEMM path moe_layer_forward takes for the workload (the library's
+    rule: block-scaled when twice the mean routed rows per expert is at most
+    64)."""
+    S = wl.T * wl.k
+    return "block-scaled" if 2 * -(-S // wl.E) <= 64 else "bf16-decode"
+
+
+def captured_traffic(workload: str):
+    rec = TRAFFIC.get(workload)
+    if rec is None or rec[0] == 0 or kernel_src_sha(rec[1]) != rec[2]:
+        return None
+    return rec[0]
 
 
 # ------------------------------------------------------------------ clocks
@@ -520,7 +538,7 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
     ms_per_step = total_ms / args.steps
     value = job_throughput(ctx.world, T, args.steps, total_ms)
 
-    # the same steps as eager calls (host planning and six launches per step)
+    # the same steps as eager calls (host planning and the launches per step)
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     for i in range(args.steps):
@@ -536,7 +554,7 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
     if layer_only:
         return {"value": value, "ms_per_step": ms_per_step, "config": config_dict(wl),
                 "launch": LAUNCH_NOTE, "eager": eager,
-                "clocks": clk, "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
+                "clocks": clk, "gpu_launches": LAUNCHES_PER_LAYER[gemm_path(wl)] * args.steps,
                 "step_ms_min": min(step_ms), "step_ms_max": max(step_ms)}
 
     # ---- roofline of the grouped expert MLP: the same step through the
@@ -575,10 +593,10 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
         roof = {"bound": "hbm", "achieved": mlp_bytes / (mlp_ms / 1e3) / 1e9, "peak": hbm,
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    traffic = TRAFFIC_BYTES.get(wl.name) if TRAFFIC_SRC_SHA == kernel_src_sha() else None
-    roof.update(traffic=traffic, kernel="moe_expert_mlp (grouped gate/up+SwiGLU and down GEMMs)",
+    roof.update(traffic=captured_traffic(wl.name),
+                kernel="moe_expert_mlp (grouped gate/up+SwiGLU and down GEMMs)",
                 algorithmic_bytes=mlp_bytes, ms=mlp_ms, peak_source=peak_kind,
-                path="block-scaled" if 2 * -(-S // E) <= 64 else "bf16-decode")
+                path=gemm_path(wl))
     layer_bytes = touched * expert_bytes(wl) + T * D * 2 + T * E * 4 + T * D * 2
     layer_flops = 6.0 * S * D * F
     t_roof_meas = max(layer_bytes / (hbm * 1e9), layer_flops / (tc_sust * 1e12))
@@ -616,7 +634,7 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
                            "frac_of_spec_8TBs_2.25PF": t_roof_spec / (ms_per_step / 1e3),
                            "touched_experts": touched},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
+        "gpu_launches": LAUNCHES_PER_LAYER[gemm_path(wl)] * args.steps,
         "wall_s_timed_region": wall, "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),
     }
 

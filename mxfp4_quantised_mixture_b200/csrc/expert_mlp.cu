@@ -36,14 +36,24 @@
 //     (token, 32-feature block), stores h to [S][F] when asked and splits it
 //     into the pieces the down GEMM reads.
 //   * down: 128 rows of the [D][F] matrix; output y_perm [S][D] bf16.
-// The kernel is persistent: one CTA per SM walks the work items (token tile,
-// weight slice) b, b + grid, ...; its copy ring (up to 12 stages of two
-// 128-K windows each, so one barrier round trip covers 256 of K) runs on
-// across items, the weight-scale block of an item is single- or
-// double-buffered and the accumulator double-buffered, so one item's
-// epilogue overlaps the next item's MMAs.
+// Both GEMMs run in one persistent launch (one CTA per SM, two for 16-token
+// tiles).  Its work items are (token tile, 128 weight rows) of the gate/up
+// GEMM, then those of the down GEMM; the CTAs take them one at a time from a
+// counter in the workspace, in index order, so an SM that finishes early
+// takes the next item, whichever GEMM it belongs to, and the down GEMM starts
+// on SMs the gate/up GEMM no longer fills.  A down item waits (bounded, on a
+// per-tile count that each gate/up item raises with release semantics after
+// its pieces of h are stored) until every gate/up item of its tile is done.
+// Every gate/up item is taken before any down item and never waits on
+// another CTA, so every such wait ends, however many CTAs are resident.
+// Each CTA's copy ring (up to 12 stages of two 128-K windows each, so one
+// barrier round trip covers 256 of K) runs on across items, the weight-scale
+// block of an item is single- or double-buffered and the accumulator
+// double-buffered, so one item's epilogue overlaps the next item's MMAs.
 // Warp roles (14 warps):
-//   warp 0      producer: per item the weight-scale bytes and the token-scale
+//   warp 0      producer: takes the work items and posts each to the other
+//               roles through a small queue in shared memory; per item the
+//               weight-scale bytes and the token-scale
 //               words (bulk copies), per 128-K window the weight codes (TMA,
 //               8 KB of packed codes that land as the 16 KB one-byte-per-code
 //               layout the MMA reads) and the token pieces (TMA, 2 NT x 128 B)
@@ -196,29 +206,92 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return r;
 }
 
-// Arguments of one GEMM launch.
+// Arguments of one GEMM of the pair: the gate/up GEMM (kind 0, input the
+// pieces of the rows, K = d_model) or the down GEMM (kind 1, input the pieces
+// of h, K = d_ff).
 struct GemmArgs {
   const uint32_t* sfx_words;  // token-scale words of the input pieces
   const uint8_t* scales;      // weight scale bytes [E][R][K/32]
+  int rows_per_expert, K, out_ld;
+  uint16_t* out;  // h (gate/up; may be null) or y_perm (down)
+};
+
+// Arguments of one launch: both GEMMs in one persistent grid.
+struct MlpArgs {
+  GemmArgs gu, dn;
   const Tile* tiles;
   const int* n_tiles;
-  int rows_per_expert, K, NS, NB, out_ld;
-  uint16_t* out;  // h (gate/up; may be null) or y_perm (down)
-  // gate/up only: the pieces of h for the down GEMM, [2 * padded rows][F]
+  int NS, NB, Kmax;
+  // written by the gate/up items: the pieces of h, [2 * padded rows][F]
   // bytes, and their scale words [tiles][F/128 windows][2 NT]
-  uint8_t* pieces_out;
-  uint32_t* words_out;
+  uint8_t* pieces_h;
+  uint32_t* words_h;
+  int* work;  // the next work item to take; zero at launch
+  int* done;  // [tiles] gate/up items finished per token tile; zero at launch
   int32_t* status;
   int fail_cta;
 };
 
-template <int NT, bool GATE_UP, bool TWO>
+// The tensor maps of both GEMMs, indexed by kind: weights (per window, the
+// moved-back last window, two windows per box) and input pieces (per
+// window, two windows per box).
+struct MlpMaps {
+  CUtensorMap w[2], wt[2], w2[2], x[2], x2[2];
+};
+
+constexpr int kQueue = 4;  // work items handed from the producer to the other roles
+constexpr int kQueueReaders = 1 + 4 + kEpiWarps;  // MMA thread, scale writers, epilogue warps
+
+// Wait until *p >= want (a count another CTA raises with release semantics),
+// then order this thread's later copies (async proxy) after what it saw.
+__device__ __forceinline__ bool wait_count(const int* p, int want, volatile int* abort,
+                                           int32_t* status) {
+  auto seen = [&]() {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v >= want;
+  };
+  bool ok = seen();
+  if (!ok) {
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+      __nanosleep(64);
+      if ((ok = seen())) break;
+      if (*abort) return false;
+      if ((i & 15u) == 0 && tc::globaltimer_ns() - t0 > kWaitLimitNs) {
+        abort_cta(abort, status);
+        return false;
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
+// One work item: kind 0 = gate/up (token tile t, 64 gate + 64 up rows at
+// feature mt * 64), kind 1 = down (tile t, 128 output rows at mt * 128).
+// Every gate/up item comes before every down item.
+struct Item {
+  int kind, t, mt;
+};
+
+__device__ __forceinline__ Item item_of(int i, int n_gu, int n_mt_gu, int n_mt_dn) {
+  Item r;
+  if (i < n_gu) {
+    r.kind = 0;
+    r.t = i / n_mt_gu;
+    r.mt = i % n_mt_gu;
+  } else {
+    r.kind = 1;
+    r.t = (i - n_gu) / n_mt_dn;
+    r.mt = (i - n_gu) % n_mt_dn;
+  }
+  return r;
+}
+
+template <int NT, bool TWO>
 __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
-    grouped_mx_gemm(const __grid_constant__ CUtensorMap map_w,
-                    const __grid_constant__ CUtensorMap map_w_tail,
-                    const __grid_constant__ CUtensorMap map_w2,
-                    const __grid_constant__ CUtensorMap map_x,
-                    const __grid_constant__ CUtensorMap map_x2, const GemmArgs args) {
+    grouped_mx_mlp(const __grid_constant__ MlpMaps maps, const MlpArgs args) {
   constexpr int XR = 2 * NT;  // token piece rows per window
   constexpr uint32_t X_BYTES = XR * BKS;
   constexpr uint32_t IDESC = tc::idesc_mx(tc::kFmtE2M1, tc::kFmtE4M3, BN, XR);
@@ -226,16 +299,16 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
   constexpr int kTmemCols = tmem_cols_for(TWO);
   static_assert(XR >= 16 && XR <= kAccCols && (X_BYTES % 1024) == 0, "token tile of 8..64 tokens");
   static_assert(!TWO || NT == 16, "two CTAs per SM only for 16-token tiles");
-  const int rows_per_expert = args.rows_per_expert, K = args.K, NS = args.NS, NB = args.NB;
+  const int NS = args.NS, NB = args.NB;
   const Tile* __restrict__ tiles = args.tiles;
   int32_t* status = args.status;
-  const int F = rows_per_expert / 2;
-  const int n_mt = GATE_UP ? (F + BN / 2 - 1) / (BN / 2) : (rows_per_expert + BN - 1) / BN;
+  const int D = args.dn.rows_per_expert, F = args.gu.rows_per_expert / 2;
+  const int n_mt_gu = (F + BN / 2 - 1) / (BN / 2), n_mt_dn = (D + BN - 1) / BN;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const SmemLayout L = smem_layout(NT, NS, NB, K);
+  const SmemLayout L = smem_layout(NT, NS, NB, args.Kmax);
   uint8_t* xs = smem + L.x_off;
   uint8_t* wsm = smem + L.w_off;
   uint8_t* aux = smem + L.a_off;
@@ -249,14 +322,14 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
   uint64_t* dempty = dfull + 2;           // [2] accumulator read by the epilogue
   uint64_t* drain = dempty + 2;           // every MMA issued has completed
   uint64_t* never = drain + 1;            // completed by nothing (the injected test wait)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(never + 1);
+  uint64_t* qfull = never + 1;            // [kQueue] work item posted
+  uint64_t* qempty = qfull + kQueue;      // [kQueue] work item read by every role
+  int* qitem = reinterpret_cast<int*>(qempty + kQueue);  // [kQueue]; -1 = no more work
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qitem + kQueue);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* prod_stages = abort_flag + 1;  // stages the producer issued (read on unwind)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwin = (K + BKS - 1) / BKS;    // 128-K windows
-  const int nstg = (nwin + WPS - 1) / WPS;  // pipeline stages of WPS windows
-  const int kscale = K / 32;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -271,16 +344,23 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
       tc::mbar_init(&dfull[a], 1);
       tc::mbar_init(&dempty[a], kEpiWarps);
     }
+    for (int q = 0; q < kQueue; ++q) {
+      tc::mbar_init(&qfull[q], 1);
+      tc::mbar_init(&qempty[q], kQueueReaders);
+    }
     tc::mbar_init(drain, 1);
     tc::mbar_init(never, 1);
     *abort_flag = 0;
     *prod_stages = 0;
     tc::fence_mbar_init();
-    tc::tma_prefetch_desc(&map_w);
-    tc::tma_prefetch_desc(&map_w_tail);
-    tc::tma_prefetch_desc(&map_w2);
-    tc::tma_prefetch_desc(&map_x);
-    tc::tma_prefetch_desc(&map_x2);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      tc::tma_prefetch_desc(&maps.w[k]);
+      tc::tma_prefetch_desc(&maps.wt[k]);
+      tc::tma_prefetch_desc(&maps.w2[k]);
+      tc::tma_prefetch_desc(&maps.x[k]);
+      tc::tma_prefetch_desc(&maps.x2[k]);
+    }
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_holder, kTmemCols);
@@ -292,42 +372,77 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t t_sf = tmem + 2 * kAccCols;  // stage slot s: columns t_sf + s * kSlotCols ...
   int my_stages = 0;  // scale writers: stages this warp has arrived on
-  // a CTA with no item runs no role loop and goes straight to the unwind
-  const int n_items = __ldg(args.n_tiles) * n_mt;
+  const int n_tiles = __ldg(args.n_tiles);
+  const int n_gu = n_tiles * n_mt_gu;
+  const int n_items = n_gu + n_tiles * n_mt_dn;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Takes the work items one at a time from the grid's counter (the next
+    // one while the current one's last two stages go out, so the atomic's
+    // round trip is hidden), posts each to the other roles, and issues its
+    // copies.  A down item first waits until every gate/up item of its tile
+    // has written its pieces of h.  Items are taken in index order, so every
+    // gate/up item is taken before any down item, and a producer never
+    // waits on another CTA while it holds a gate/up item: the wait always
+    // ends.
     if (lane == 0) {
       int g = 0, it = 0;
       int s_slot = 0;          // ring slot of stage g
       uint32_t s_phase = 0;    // parity of slot s_slot's current use
-      bool ok = true;
-      for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
-        const int t = i / n_mt, mt = i % n_mt;
-        const Tile tile = tiles[t];
+      int next = 0;
+      bool taken = false;      // next holds an item already taken
+      for (;;) {
+        const int qs = it % kQueue;
+        if (it >= kQueue && !wait1(&qempty[qs], ((it / kQueue) - 1) & 1, abort_flag, status)) break;
         const int b = it % NB, use = it / NB;
         // the auxiliary buffer is free once the scale writers are done with its last item
         if (use > 0 && !wait1(&sfree[b], (use - 1) & 1, abort_flag, status)) break;
+        const int i = taken ? next : atomicAdd(args.work, 1);
+        taken = false;
+        qitem[qs] = i < n_items ? i : -1;
+        tc::mbar_arrive(&qfull[qs]);
+        if (i >= n_items) break;
+        const Item I = item_of(i, n_gu, n_mt_gu, n_mt_dn);
+        const bool gu = I.kind == 0;
+        if (!gu && !wait_count(args.done + I.t, n_mt_gu, abort_flag, status)) break;
+        const int K = gu ? args.gu.K : args.dn.K;
+        const int rows_per_expert = gu ? args.gu.rows_per_expert : args.dn.rows_per_expert;
+        const uint8_t* scales = gu ? args.gu.scales : args.dn.scales;
+        const uint32_t* sfx_words = gu ? args.gu.sfx_words : args.dn.sfx_words;
+        const int nwin = (K + BKS - 1) / BKS, nstg = (nwin + WPS - 1) / WPS, kscale = K / 32;
+        const CUtensorMap* mw = &maps.w[I.kind];
+        const CUtensorMap* mwt = &maps.wt[I.kind];
+        const CUtensorMap* mw2 = &maps.w2[I.kind];
+        const CUtensorMap* mx = &maps.x[I.kind];
+        const CUtensorMap* mx2 = &maps.x2[I.kind];
+        const Tile tile = tiles[I.t];
         const int64_t erow = static_cast<int64_t>(tile.e) * rows_per_expert;
         uint8_t* sdst = aux + b * L.aux_bytes;
         const uint32_t wbytes = static_cast<uint32_t>(nwin) * XR * 4;
-        if (GATE_UP) {
-          const int f0 = mt * (BN / 2);
+        if (gu) {
+          const int f0 = I.mt * (BN / 2);
           const uint32_t bytes = static_cast<uint32_t>(min(BN / 2, F - f0)) * kscale;
           tc::mbar_arrive_expect_tx(&sbar[b], 2 * bytes + wbytes);
-          tc::bulk_load(sdst, args.scales + (erow + f0) * kscale, bytes, &sbar[b]);
-          tc::bulk_load(sdst + (BN / 2) * kscale, args.scales + (erow + F + f0) * kscale, bytes,
+          tc::bulk_load(sdst, scales + (erow + f0) * kscale, bytes, &sbar[b]);
+          tc::bulk_load(sdst + (BN / 2) * kscale, scales + (erow + F + f0) * kscale, bytes,
                         &sbar[b]);
         } else {
-          const int d0 = mt * BN;
+          const int d0 = I.mt * BN;
           const uint32_t bytes = static_cast<uint32_t>(min(BN, rows_per_expert - d0)) * kscale;
           tc::mbar_arrive_expect_tx(&sbar[b], bytes + wbytes);
-          tc::bulk_load(sdst, args.scales + (erow + d0) * kscale, bytes, &sbar[b]);
+          tc::bulk_load(sdst, scales + (erow + d0) * kscale, bytes, &sbar[b]);
         }
-        tc::bulk_load(sdst + L.wsc_bytes, args.sfx_words + static_cast<int64_t>(t) * nwin * XR,
+        tc::bulk_load(sdst + L.wsc_bytes, sfx_words + static_cast<int64_t>(I.t) * nwin * XR,
                       wbytes, &sbar[b]);
-        const int wrow = GATE_UP ? mt * (BN / 2) : mt * BN;
+        ++it;  // items whose auxiliary copies were issued
+        const int wrow = gu ? I.mt * (BN / 2) : I.mt * BN;
+        bool ok = true;
         for (int st = 0; st < nstg; ++st, ++g) {
+          if (st == (nstg >= 2 ? nstg - 2 : 0)) {
+            next = atomicAdd(args.work, 1);
+            taken = true;
+          }
           if (g >= NS && !wait1(&empty[s_slot], s_phase ^ 1u, abort_flag, status)) {
             ok = false;
             break;
@@ -339,36 +454,37 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
             // two whole windows: one copy of each operand for the stage (the
             // copy engine's cost is mostly per copy, not per byte)
             uint8_t* wdst = wsm + s_slot * WPS * W_SMEM;
-            if (GATE_UP) {
-              tc::tma_load_5d(wdst, &map_w2, &full[s_slot], 0, 0, wrow, w0, tile.e);
+            if (gu) {
+              tc::tma_load_5d(wdst, mw2, &full[s_slot], 0, 0, wrow, w0, tile.e);
             } else {
-              tc::tma_load_4d(wdst, &map_w2, &full[s_slot], 0, wrow, w0, tile.e);
+              tc::tma_load_4d(wdst, mw2, &full[s_slot], 0, wrow, w0, tile.e);
             }
-            tc::tma_load_3d(xs + s_slot * WPS * X_BYTES, &map_x2, &full[s_slot], 0, t * XR, w0);
+            tc::tma_load_3d(xs + s_slot * WPS * X_BYTES, mx2, &full[s_slot], 0, I.t * XR, w0);
           } else for (int v = 0; v < nv; ++v) {
             const int w = w0 + v;
             const int k0 = stage_k0(w, K);
             uint8_t* wdst = wsm + (s_slot * WPS + v) * W_SMEM;
             if (k0 == w * BKS) {
-              if (GATE_UP) {
-                tc::tma_load_5d(wdst, &map_w, &full[s_slot], 0, w, 0, wrow, tile.e);
+              if (gu) {
+                tc::tma_load_5d(wdst, mw, &full[s_slot], 0, w, 0, wrow, tile.e);
               } else {
-                tc::tma_load_4d(wdst, &map_w, &full[s_slot], 0, w, wrow, tile.e);
+                tc::tma_load_4d(wdst, mw, &full[s_slot], 0, w, wrow, tile.e);
               }
             } else {
-              if (GATE_UP) {
-                tc::tma_load_4d(wdst, &map_w_tail, &full[s_slot], 0, 0, wrow, tile.e);
+              if (gu) {
+                tc::tma_load_4d(wdst, mwt, &full[s_slot], 0, 0, wrow, tile.e);
               } else {
-                tc::tma_load_3d(wdst, &map_w_tail, &full[s_slot], 0, wrow, tile.e);
+                tc::tma_load_3d(wdst, mwt, &full[s_slot], 0, wrow, tile.e);
               }
             }
-            tc::tma_load_2d(xs + (s_slot * WPS + v) * X_BYTES, &map_x, &full[s_slot], k0, t * XR);
+            tc::tma_load_2d(xs + (s_slot * WPS + v) * X_BYTES, mx, &full[s_slot], k0, I.t * XR);
           }
           if (++s_slot == NS) {
             s_slot = 0;
             s_phase ^= 1u;
           }
         }
+        if (!ok) break;
       }
       *prod_stages = g;
       // the items whose auxiliary copies were issued: [it - NB, it) at most
@@ -387,7 +503,6 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
       bool ok = true, any = false;
       const uint64_t xdesc0 = tc::smem_desc_sw128(tc::smem_u32(xs));
       const uint64_t wdesc0 = tc::smem_desc_sw128(tc::smem_u32(wsm));
-      const int tail_w = (K % BKS) ? nwin - 1 : nwin;  // the re-read window, if any
       // testing only: the first wait of this CTA waits on a barrier that
       // nothing completes, with a short limit, and gives up as a timeout would
       if (static_cast<int>(blockIdx.x) == args.fail_cta &&
@@ -395,7 +510,15 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
         abort_cta(abort_flag, status);
         ok = false;
       }
-      for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++it) {
+      for (; ok; ++it) {
+        const int qs = it % kQueue;
+        if (!wait1(&qfull[qs], (it / kQueue) & 1, abort_flag, status)) break;
+        const int i = qitem[qs];
+        tc::mbar_arrive(&qempty[qs]);
+        if (i < 0) break;
+        const int K = i < n_gu ? args.gu.K : args.dn.K;
+        const int nwin = (K + BKS - 1) / BKS, nstg = (nwin + WPS - 1) / WPS;
+        const int tail_w = (K % BKS) ? nwin - 1 : nwin;  // the re-read window, if any
         const uint32_t d = tmem + (it & 1) * kAccCols;
         // accumulator it & 1 was last used by item it - 2
         if (it >= 2) {
@@ -456,8 +579,18 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
     int g = 0, it = 0;
     int s_slot = 0;        // stage slot (and scale slot) of stage g
     uint32_t s_phase = 0;  // parity of its current use
-    for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++it) {
-      const int mt = i % n_mt;
+    for (;; ++it) {
+      const int qs = it % kQueue;
+      if (!warp_wait(&qfull[qs], (it / kQueue) & 1, abort_flag, status, 64)) break;
+      const int i = qitem[qs];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&qempty[qs]);
+      if (i < 0) break;
+      const Item I = item_of(i, n_gu, n_mt_gu, n_mt_dn);
+      const bool gu = I.kind == 0;
+      const int K = gu ? args.gu.K : args.dn.K;
+      const int nwin = (K + BKS - 1) / BKS, nstg = (nwin + WPS - 1) / WPS, kscale = K / 32;
+      const int mt = I.mt;
       const int b = it % NB;
       if (!warp_wait(&sbar[b], (it / NB) & 1, abort_flag, status, 64)) break;
       const uint8_t* sblock = aux + b * L.aux_bytes;
@@ -468,12 +601,12 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int n = 32 * c + lane;
-        if (GATE_UP) {
+        if (gu) {
           srow[c] = (n & 1) * (BN / 2) + (n >> 1);
           live[c] = mt * (BN / 2) + (n >> 1) < F;
         } else {
           srow[c] = n;
-          live[c] = mt * BN + n < rows_per_expert;
+          live[c] = mt * BN + n < D;
         }
       }
       const uint8_t* wsc[4];
@@ -535,17 +668,27 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
     // ------------------------------------------------------------ epilogue
     // Lane l of quarter q holds weight row m = 32 q + l of the item; this
     // warp reads the accumulator columns of tokens [half HT, half HT + HT).
+    // The eight warps leave the loop only together (after a barrier that all
+    // of them reach), so none is left waiting at one of their barriers.
     constexpr int HT = NT / 2;
     const int q = warp & 3;
     const int half = (warp - 6) >> 2;
     const int ew = warp - 6;  // epilogue warp 0..7
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    int it = 0;
-    for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++it) {
-      const int t = i / n_mt, mt = i % n_mt;
-      const Tile tile = tiles[t];
+    for (int it = 0;; ++it) {
+      const int qs = it % kQueue;
+      bool ok = warp_wait(&qfull[qs], (it / kQueue) & 1, abort_flag, status, 256);
+      int i = -1;
+      if (ok) {
+        i = qitem[qs];
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&qempty[qs]);
+      }
+      if (!tc::bar_and(1, 32 * kEpiWarps, ok) || i < 0) break;
+      const Item I = item_of(i, n_gu, n_mt_gu, n_mt_dn);
+      const Tile tile = tiles[I.t];
       const int a = it & 1;
-      const bool ok = warp_wait(&dfull[a], (it >> 1) & 1, abort_flag, status, 256);
+      ok = warp_wait(&dfull[a], (it >> 1) & 1, abort_flag, status, 256);
       float acc[HT];  // token half HT + j of this lane's row: hi + lo piece
       if (ok) {
         tc::tc_fence_after();
@@ -564,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&dempty[a]);
       }
-      if (GATE_UP) {
+      if (I.kind == 0) {
         // lanes 2j (gate) and 2j + 1 (up) hold local feature fl = 16 q + j;
         // the gate lane finishes the first HT / 2 tokens, the up lane the rest
         constexpr int QT = HT / 2;
@@ -581,28 +724,27 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
             hs[(half * HT + (up ? QT : 0) + j) * (BN / 2) + fl] = f32_to_bf16_rne(hh);
           }
         }
-        // every epilogue warp takes part (a failed wait included), so the
-        // barrier cannot strand one; all leave together if any failed
         if (!tc::bar_and(1, 32 * kEpiWarps, ok)) break;
         // one warp per (token, 32-feature block): store h, split it into the
         // pieces of the down GEMM and write the block's scale bytes
-        const int fb0 = mt * (BN / 2);
+        const int fb0 = I.mt * (BN / 2);
         const int nunits = tile.nrows * 2;
         for (int u = ew; u < nunits; u += kEpiWarps) {
           const int tl = u >> 1, b = u & 1;
           const int f = fb0 + 32 * b + lane;
           const uint16_t hbits = hs[tl * (BN / 2) + 32 * b + lane];
           const float v = bf16_to_f32(hbits);
-          if (args.out) args.out[static_cast<int64_t>(tile.row0 + tl) * args.out_ld + f] = hbits;
+          if (args.gu.out)
+            args.gu.out[static_cast<int64_t>(tile.row0 + tl) * args.gu.out_ld + f] = hbits;
           float amax = fabsf(v);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
           const int te = split_exponent(amax);
           uint8_t hi, lo;
           split1(v, te, hi, lo);
-          const int64_t p = static_cast<int64_t>(t) * NT + tl;  // padded row of this token
-          args.pieces_out[(2 * p) * F + f] = hi;
-          args.pieces_out[(2 * p + 1) * F + f] = lo;
+          const int64_t p = static_cast<int64_t>(I.t) * NT + tl;  // padded row of this token
+          args.pieces_h[(2 * p) * F + f] = hi;
+          args.pieces_h[(2 * p + 1) * F + f] = lo;
           if (lane == 0) {
             // scale bytes of block blk in the words of the window(s) that
             // cover it: window blk / 4 (byte blk % 4), and, when F is not a
@@ -612,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
             const int tail0 = (F % BKS) ? (F - BKS) / 32 : 0x7FFFFFFF;
             auto put = [&](int w, int byte) {
               uint8_t* wb = reinterpret_cast<uint8_t*>(
-                  args.words_out + (static_cast<int64_t>(t) * nwo + w) * (2 * NT) + 2 * tl);
+                  args.words_h + (static_cast<int64_t>(I.t) * nwo + w) * (2 * NT) + 2 * tl);
               wb[byte] = static_cast<uint8_t>(te + 127);
               wb[4 + byte] = static_cast<uint8_t>(te + 123);
             };
@@ -620,15 +762,22 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
             if (blk >= tail0) put(nwo - 1, blk - tail0);
           }
         }
-      } else {
-        if (!ok) break;
-        const int dd = mt * BN + 32 * q + lane;
-        if (dd < rows_per_expert) {
-          uint16_t* ocol = args.out + static_cast<int64_t>(tile.row0) * args.out_ld + dd;
+        // every store of this item is done: release it to the tile's down
+        // items (read by copies in other CTAs)
+        tc::bar_and(1, 32 * kEpiWarps, true);
+        if (ew == 0 && lane == 0) {
+          __threadfence();
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(args.done + I.t) : "memory");
+        }
+      } else if (ok) {
+        const int dd = I.mt * BN + 32 * q + lane;
+        if (dd < D) {
+          uint16_t* ocol = args.dn.out + static_cast<int64_t>(tile.row0) * args.dn.out_ld + dd;
 #pragma unroll
           for (int j = 0; j < HT; ++j) {
             const int tl = half * HT + j;
-            if (tl < tile.nrows) ocol[static_cast<int64_t>(tl) * args.out_ld] = f32_to_bf16_rne(acc[j]);
+            if (tl < tile.nrows) ocol[static_cast<int64_t>(tl) * args.dn.out_ld] = f32_to_bf16_rne(acc[j]);
           }
         }
       }
@@ -676,7 +825,13 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
 __global__ void __launch_bounds__(256) split_rows_kernel(
     const uint16_t* __restrict__ src, const int32_t* __restrict__ gather, int k, int K,
     const Tile* __restrict__ tiles, const int* __restrict__ n_tiles, int NT, int64_t padded_rows,
-    uint8_t* __restrict__ pieces, uint32_t* __restrict__ words) {
+    uint8_t* __restrict__ pieces, uint32_t* __restrict__ words, int* __restrict__ work,
+    int* __restrict__ done, int n_done) {
+  // the work counter and the per-tile counts of the GEMM launch that follows
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    for (int j = threadIdx.x; j < n_done; j += blockDim.x) done[j] = 0;
+    if (threadIdx.x == 0) *work = 0;
+  }
   const int nstg = (K + BKS - 1) / BKS;
   const int st = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -859,52 +1014,46 @@ bool allow_smem(Kern kern, std::atomic<uint64_t>& done) {
   return true;
 }
 
-template <int NT, bool GATE_UP, bool TWO>
-bool prepare_gemm() {
+template <int NT, bool TWO>
+bool prepare_mlp() {
   static std::atomic<uint64_t> done{0};
-  return allow_smem(grouped_mx_gemm<NT, GATE_UP, TWO>, done);
+  return allow_smem(grouped_mx_mlp<NT, TWO>, done);
 }
 
 bool prepare_nt(int NT, int CPS) {
   switch (NT) {
     case 16:
-      return CPS == 2 ? prepare_gemm<16, true, true>() && prepare_gemm<16, false, true>()
-                      : prepare_gemm<16, true, false>() && prepare_gemm<16, false, false>();
+      return CPS == 2 ? prepare_mlp<16, true>() : prepare_mlp<16, false>();
     case 32:
-      return prepare_gemm<32, true, false>() && prepare_gemm<32, false, false>();
+      return prepare_mlp<32, false>();
     default:
-      return prepare_gemm<64, true, false>() && prepare_gemm<64, false, false>();
+      return prepare_mlp<64, false>();
   }
 }
 
-template <int NT, bool GATE_UP, bool TWO>
-moe_status launch_gemm(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& mwt,
-                       const CUtensorMap& mw2, const CUtensorMap& mx, const CUtensorMap& mx2,
-                       const GemmArgs& a, int max_items,
-                       cudaStream_t stream) {
-  const int smem = smem_bytes(NT, P.NS, P.NB, a.K);
+template <int NT, bool TWO>
+moe_status launch_mlp(const MxPlan& P, const MlpMaps& maps, const MlpArgs& a, int max_items,
+                      cudaStream_t stream) {
+  const int smem = smem_bytes(NT, P.NS, P.NB, a.Kmax);
   const int slots = (TWO ? 2 : 1) * sm_count();
   const int grid = max_items < slots ? max_items : slots;
   // one CTA per SM holds all 512 tensor-memory columns: it asks for enough
   // shared memory that no second CTA shares the SM
   const int smem_launch =
       TWO || smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
-  return launch(grouped_mx_gemm<NT, GATE_UP, TWO>, dim3(grid), dim3(kThreads), smem_launch,
-                stream, mw, mwt, mw2, mx, mx2, a);
+  return launch(grouped_mx_mlp<NT, TWO>, dim3(grid), dim3(kThreads), smem_launch, stream, maps, a);
 }
 
-template <bool GATE_UP>
-moe_status launch_nt(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& mwt,
-                     const CUtensorMap& mw2, const CUtensorMap& mx, const CUtensorMap& mx2,
-                     const GemmArgs& a, int max_items, cudaStream_t st) {
+moe_status launch_nt(const MxPlan& P, const MlpMaps& maps, const MlpArgs& a, int max_items,
+                     cudaStream_t st) {
   switch (P.NT) {
     case 16:
-      return P.CPS == 2 ? launch_gemm<16, GATE_UP, true>(P, mw, mwt, mw2, mx, mx2, a, max_items, st)
-                        : launch_gemm<16, GATE_UP, false>(P, mw, mwt, mw2, mx, mx2, a, max_items, st);
+      return P.CPS == 2 ? launch_mlp<16, true>(P, maps, a, max_items, st)
+                        : launch_mlp<16, false>(P, maps, a, max_items, st);
     case 32:
-      return launch_gemm<32, GATE_UP, false>(P, mw, mwt, mw2, mx, mx2, a, max_items, st);
+      return launch_mlp<32, false>(P, maps, a, max_items, st);
     default:
-      return launch_gemm<64, GATE_UP, false>(P, mw, mwt, mw2, mx, mx2, a, max_items, st);
+      return launch_mlp<64, false>(P, maps, a, max_items, st);
   }
 }
 
@@ -912,7 +1061,7 @@ moe_status launch_nt(const MxPlan& P, const CUtensorMap& mw, const CUtensorMap& 
 // and for h each its pieces [2 * padded rows][K] and scale words
 // [tiles][K/128 windows][2 NT].
 struct MxWs {
-  size_t n_tiles, tiles, pieces_x, words_x, pieces_h, words_h, total;
+  size_t n_tiles, tiles, pieces_x, words_x, pieces_h, words_h, sched, total;
   int64_t max_tiles, padded_rows;
 };
 
@@ -932,7 +1081,8 @@ MxWs mx_ws(const moe_shape& sh) {
   w.words_x = align_up(w.pieces_x + 2 * static_cast<size_t>(w.padded_rows) * D, 256);
   w.pieces_h = align_up(w.words_x + words_bytes(D), 256);
   w.words_h = align_up(w.pieces_h + 2 * static_cast<size_t>(w.padded_rows) * F, 256);
-  w.total = align_up(w.words_h + words_bytes(F), 256);
+  w.sched = align_up(w.words_h + words_bytes(F), 256);  // work counter, then [max tiles] counts
+  w.total = align_up(w.sched + (1 + static_cast<size_t>(w.max_tiles)) * sizeof(int), 256);
   return w;
 }
 
@@ -960,6 +1110,8 @@ moe_status mx_plan(MlpPlan* p, void* ws) {
   P.words_x = reinterpret_cast<uint32_t*>(base + W.words_x);
   P.pieces_h = reinterpret_cast<uint8_t*>(base + W.pieces_h);
   P.words_h = reinterpret_cast<uint32_t*>(base + W.words_h);
+  P.work = reinterpret_cast<int*>(base + W.sched);
+  P.done = P.work + 1;
   const int D = sh.d_model, F = sh.d_ff, E = sh.E;
   if (!make_weight_maps(&P.m_gu, &P.m_gu_t, &P.m_gu2, p->wgu_q, E, 2 * F, D, true) ||
       !make_weight_maps(&P.m_dn, &P.m_dn_t, &P.m_dn2, p->wdn_q, E, D, F, false) ||
@@ -989,40 +1141,51 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
                 from_x ? in.x : p.x_perm,
                 from_x ? in.sorted_slot : static_cast<const int32_t*>(nullptr), from_x ? in.k : 1,
                 D, static_cast<const Tile*>(p.tiles), static_cast<const int*>(p.n_tiles), NT,
-                P.padded_rows, P.pieces_x, P.words_x);
+                P.padded_rows, P.pieces_x, P.words_x, P.work, P.done,
+                static_cast<int>(P.max_tiles));
     if (st != MOE_OK) return st;
   }
   const int max_tiles = static_cast<int>(P.max_tiles);
   const int mt_gu = (F + BN / 2 - 1) / (BN / 2), mt_dn = (D + BN - 1) / BN;
-  GemmArgs a{};
+  MlpMaps maps;
+  maps.w[0] = P.m_gu;
+  maps.wt[0] = P.m_gu_t;
+  maps.w2[0] = P.m_gu2;
+  maps.x[0] = P.m_x;
+  maps.x2[0] = P.m_x2;
+  maps.w[1] = P.m_dn;
+  maps.wt[1] = P.m_dn_t;
+  maps.w2[1] = P.m_dn2;
+  maps.x[1] = P.m_h;
+  maps.x2[1] = P.m_h2;
+  MlpArgs a{};
   a.tiles = p.tiles;
   a.n_tiles = p.n_tiles;
   a.NS = P.NS;
   a.NB = P.NB;
-  a.status = status;
+  a.Kmax = D > F ? D : F;
   // gate/up + SwiGLU: h (when asked) and the pieces of h
-  a.sfx_words = P.words_x;
-  a.scales = p.wgu_s;
-  a.rows_per_expert = 2 * F;
-  a.K = D;
-  a.out_ld = F;
-  a.out = p.h;
-  a.pieces_out = P.pieces_h;
-  a.words_out = P.words_h;
-  a.fail_cta = fail_cta;
-  if ((st = launch_nt<true>(P, P.m_gu, P.m_gu_t, P.m_gu2, P.m_x, P.m_x2, a, max_tiles * mt_gu, stream)) != MOE_OK)
-    return st;
+  a.gu.sfx_words = P.words_x;
+  a.gu.scales = p.wgu_s;
+  a.gu.rows_per_expert = 2 * F;
+  a.gu.K = D;
+  a.gu.out_ld = F;
+  a.gu.out = p.h;
+  a.pieces_h = P.pieces_h;
+  a.words_h = P.words_h;
   // down
-  a.sfx_words = P.words_h;
-  a.scales = p.wdn_s;
-  a.rows_per_expert = D;
-  a.K = F;
-  a.out_ld = D;
-  a.out = p.y_perm;
-  a.pieces_out = nullptr;
-  a.words_out = nullptr;
-  a.fail_cta = -1;
-  return launch_nt<false>(P, P.m_dn, P.m_dn_t, P.m_dn2, P.m_h, P.m_h2, a, max_tiles * mt_dn, stream);
+  a.dn.sfx_words = P.words_h;
+  a.dn.scales = p.wdn_s;
+  a.dn.rows_per_expert = D;
+  a.dn.K = F;
+  a.dn.out_ld = D;
+  a.dn.out = p.y_perm;
+  a.work = P.work;
+  a.done = P.done;
+  a.status = status;
+  a.fail_cta = fail_cta;
+  (void)E;
+  return launch_nt(P, maps, a, max_tiles * (mt_gu + mt_dn), stream);
 }
 
 }  // namespace moe

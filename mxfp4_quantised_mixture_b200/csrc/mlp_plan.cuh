@@ -53,6 +53,8 @@ struct MxPlan {
   int64_t max_tiles, padded_rows;
   uint8_t *pieces_x, *pieces_h;
   uint32_t *words_x, *words_h;
+  int* work;  // the GEMM launch's work counter, then its per-tile counts [max_tiles]
+  int* done;
 };
 
 // Decode-to-bf16 path (csrc/expert_mlp_bf16.cu)

@@ -1,13 +1,16 @@
 """The bounded-wait failure path of both grouped GEMMs, without a GPU fault.
 
 moe_expert_mlp_ex(test_timeout_cta=0) makes the first pipeline wait of the
-MMA issuer in CTA 0 of the first GEMM wait on a barrier that nothing
+MMA issuer in CTA 0 of the (first) GEMM launch wait on a barrier that nothing
 completes, with a short limit, so it gives up as a real timeout would: the
 CTA records MOE_ERR_TIMEOUT in the device status word, every role leaves its
 loop, the CTA waits for its own copies and MMAs to finish (the drains do not
-look at the abort flag), frees its tensor memory and exits; the other CTAs
-finish normally.  The host reads the status after a sync and the context
-stays usable: the next normal call gives the earlier result bit for bit.
+look at the abort flag), frees its tensor memory and exits.  The other CTAs
+finish their work; on the block-scaled path, where one launch runs both
+GEMMs, a CTA whose down item needs a gate/up item that CTA 0 took and left
+undone gives up the same way after the wait limit.  The host reads the status
+after a sync and the context stays usable: the next normal call gives the
+earlier result bit for bit.
 """
 import numpy as np
 import pytest
