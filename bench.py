@@ -88,8 +88,8 @@ TRAFFIC: dict[str, tuple[int, str, str]] = {
     "120b_skewed_prefill": (615571200 + 381615104 + 496563968 + 374050048,
                             "expert_mlp_bf16.cu", "b96e9f861b69c97f"),
     # the one launch of both GEMMs
-    "120b_decode": (0, "expert_mlp.cu", "MX_SHA"),
-    "20b_decode": (0, "expert_mlp.cu", "MX_SHA"),
+    "120b_decode": (1609689856 + 11472896, "expert_mlp.cu", "677cfa72aae5d735"),
+    "20b_decode": (429354496 + 5372928, "expert_mlp.cu", "677cfa72aae5d735"),
 }
 
 
