@@ -18,7 +18,7 @@ moe_status route_launch(const float* logits, int T, int E, int k, int32_t* idx, 
 moe_status permute_launch(const int32_t* idx, const uint16_t* x, const moe_shape& sh,
                           int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
                           int32_t* slot_pos, uint16_t* x_perm, int NT, Tile* tiles,
-                          int* n_tiles, cudaStream_t stream);
+                          int* n_tiles, int* sched, int n_sched, cudaStream_t stream);
 moe_status combine_launch(const uint16_t* y_perm, const int32_t* slot_pos, const float* w,
                           const moe_shape& sh, uint16_t* out, cudaStream_t stream);
 size_t unquantised_workspace(const moe_shape& sh);
@@ -266,7 +266,8 @@ moe_status moe_layer_forward(const uint16_t* x, const float* logits, moe_shape s
   if ((st = route_launch(logits, shape.T, shape.E, shape.k, idx, w, status, s)) != MOE_OK)
     return st;
   if ((st = permute_launch(idx, x, shape, counts, offsets, sorted_slot, slot_pos,
-                           block_scaled ? nullptr : x_perm, NT, plan.tiles, plan.n_tiles, s)) != MOE_OK)
+                           block_scaled ? nullptr : x_perm, NT, plan.tiles, plan.n_tiles,
+                           plan.sched, plan.n_sched, s)) != MOE_OK)
     return st;
   MlpInput in{};
   in.offsets = offsets;

@@ -56,20 +56,48 @@ int sm_count();
 
 bool shape_ok(const moe_shape& s);
 
-// Launch a kernel with cudaLaunchKernelEx (argument coercion as for <<< >>>).
+// Launch a kernel with cudaLaunchKernelEx (argument coercion as for <<< >>>);
+// with `early`, the kernel may start while the kernel before it on
+// the stream still runs (once every CTA of that kernel has executed
+// allow_dependents()).  Such a kernel must call wait_for_previous() before it
+// reads anything the previous kernel writes; whatever the kernels before
+// that one wrote is visible from its start.
 template <typename... Params, typename... Args>
-moe_status launch(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
-                  cudaStream_t stream, Args&&... args) {
+moe_status launch_ex(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t stream, bool early, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = early ? attr : nullptr;
+  cfg.numAttrs = early ? 1 : 0;
   if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+
+// Launch a kernel with cudaLaunchKernelEx (argument coercion as for <<< >>>),
+// in plain stream order.
+template <typename... Params, typename... Args>
+moe_status launch(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                  cudaStream_t stream, Args&&... args) {
+  return launch_ex(kern, grid, block, smem, stream, false, std::forward<Args>(args)...);
+}
+
+// Device side of launch_ex: let the next kernel on the stream start, and
+// wait until the previous kernel has completed with its writes visible (a
+// no-op when this kernel was not launched early).
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_for_previous() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace moe

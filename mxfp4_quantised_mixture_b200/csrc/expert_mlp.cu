@@ -392,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
       uint32_t s_phase = 0;    // parity of slot s_slot's current use
       int next = 0;
       bool taken = false;      // next holds an item already taken
+      bool dep = false;        // waited for the split kernel before this launch
       for (;;) {
         const int qs = it % kQueue;
         if (it >= kQueue && !wait1(&qempty[qs], ((it / kQueue) - 1) & 1, abort_flag, status)) break;
@@ -433,13 +434,87 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
           tc::mbar_arrive_expect_tx(&sbar[b], bytes + wbytes);
           tc::bulk_load(sdst, scales + (erow + d0) * kscale, bytes, &sbar[b]);
         }
-        tc::bulk_load(sdst + L.wsc_bytes, sfx_words + static_cast<int64_t>(I.t) * nwin * XR,
-                      wbytes, &sbar[b]);
+        // the first gate/up item of this CTA: its token side (pieces and
+        // words, written by the split kernel) waits for that kernel, its
+        // weights do not
+        const bool early = gu && !dep;
+        if (!early)
+          tc::bulk_load(sdst + L.wsc_bytes, sfx_words + static_cast<int64_t>(I.t) * nwin * XR,
+                        wbytes, &sbar[b]);
         ++it;  // items whose auxiliary copies were issued
         const int wrow = gu ? I.mt * (BN / 2) : I.mt * BN;
+        const int take_at = nstg >= 2 ? nstg - 2 : 0;
+        // stage st into ring slot `slot`: the barrier's byte count and the
+        // weight copies, then the token copies
+        auto issue_w = [&](int st, int slot) {
+          const int w0 = st * WPS;
+          const int nv = min(WPS, nwin - w0);
+          tc::mbar_arrive_expect_tx(&full[slot], nv * (W_TX + X_BYTES));
+          if (nv == 2 && w0 + 1 < K / BKS) {
+            // two whole windows: one copy of each operand for the stage (the
+            // copy engine's cost is mostly per copy, not per byte)
+            uint8_t* wdst = wsm + slot * WPS * W_SMEM;
+            if (gu) {
+              tc::tma_load_5d(wdst, mw2, &full[slot], 0, 0, wrow, w0, tile.e);
+            } else {
+              tc::tma_load_4d(wdst, mw2, &full[slot], 0, wrow, w0, tile.e);
+            }
+          } else {
+            for (int v = 0; v < nv; ++v) {
+              const int w = w0 + v;
+              uint8_t* wdst = wsm + (slot * WPS + v) * W_SMEM;
+              if (stage_k0(w, K) == w * BKS) {
+                if (gu) {
+                  tc::tma_load_5d(wdst, mw, &full[slot], 0, w, 0, wrow, tile.e);
+                } else {
+                  tc::tma_load_4d(wdst, mw, &full[slot], 0, w, wrow, tile.e);
+                }
+              } else {
+                if (gu) {
+                  tc::tma_load_4d(wdst, mwt, &full[slot], 0, 0, wrow, tile.e);
+                } else {
+                  tc::tma_load_3d(wdst, mwt, &full[slot], 0, wrow, tile.e);
+                }
+              }
+            }
+          }
+        };
+        auto issue_x = [&](int st, int slot) {
+          const int w0 = st * WPS;
+          const int nv = min(WPS, nwin - w0);
+          if (nv == 2 && w0 + 1 < K / BKS) {
+            tc::tma_load_3d(xs + slot * WPS * X_BYTES, mx2, &full[slot], 0, I.t * XR, w0);
+          } else {
+            for (int v = 0; v < nv; ++v)
+              tc::tma_load_2d(xs + (slot * WPS + v) * X_BYTES, mx, &full[slot],
+                              stage_k0(w0 + v, K), I.t * XR);
+          }
+        };
+        int st0 = 0;
+        if (early) {
+          // on this CTA's first item the first NS stages need no free slot:
+          // their weights go out before the wait
+          const int pre = g == 0 ? min(NS, nstg) : 0;
+          for (int st = 0; st < pre; ++st) {
+            if (st == take_at) {
+              next = atomicAdd(args.work, 1);
+              taken = true;
+            }
+            issue_w(st, st);
+          }
+          wait_for_previous();
+          dep = true;
+          tc::bulk_load(sdst + L.wsc_bytes, sfx_words + static_cast<int64_t>(I.t) * nwin * XR,
+                        wbytes, &sbar[b]);
+          for (int st = 0; st < pre; ++st) issue_x(st, st);
+          st0 = pre;
+          g += pre;
+          s_slot = pre % NS;
+          s_phase = pre == NS ? 1u : 0u;
+        }
         bool ok = true;
-        for (int st = 0; st < nstg; ++st, ++g) {
-          if (st == (nstg >= 2 ? nstg - 2 : 0)) {
+        for (int st = st0; st < nstg; ++st, ++g) {
+          if (st == take_at) {
             next = atomicAdd(args.work, 1);
             taken = true;
           }
@@ -447,38 +522,8 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
             ok = false;
             break;
           }
-          const int w0 = st * WPS;
-          const int nv = min(WPS, nwin - w0);
-          tc::mbar_arrive_expect_tx(&full[s_slot], nv * (W_TX + X_BYTES));
-          if (nv == 2 && w0 + 1 < K / BKS) {
-            // two whole windows: one copy of each operand for the stage (the
-            // copy engine's cost is mostly per copy, not per byte)
-            uint8_t* wdst = wsm + s_slot * WPS * W_SMEM;
-            if (gu) {
-              tc::tma_load_5d(wdst, mw2, &full[s_slot], 0, 0, wrow, w0, tile.e);
-            } else {
-              tc::tma_load_4d(wdst, mw2, &full[s_slot], 0, wrow, w0, tile.e);
-            }
-            tc::tma_load_3d(xs + s_slot * WPS * X_BYTES, mx2, &full[s_slot], 0, I.t * XR, w0);
-          } else for (int v = 0; v < nv; ++v) {
-            const int w = w0 + v;
-            const int k0 = stage_k0(w, K);
-            uint8_t* wdst = wsm + (s_slot * WPS + v) * W_SMEM;
-            if (k0 == w * BKS) {
-              if (gu) {
-                tc::tma_load_5d(wdst, mw, &full[s_slot], 0, w, 0, wrow, tile.e);
-              } else {
-                tc::tma_load_4d(wdst, mw, &full[s_slot], 0, w, wrow, tile.e);
-              }
-            } else {
-              if (gu) {
-                tc::tma_load_4d(wdst, mwt, &full[s_slot], 0, 0, wrow, tile.e);
-              } else {
-                tc::tma_load_3d(wdst, mwt, &full[s_slot], 0, wrow, tile.e);
-              }
-            }
-            tc::tma_load_2d(xs + (s_slot * WPS + v) * X_BYTES, mx, &full[s_slot], k0, I.t * XR);
-          }
+          issue_w(st, s_slot);
+          issue_x(st, s_slot);
           if (++s_slot == NS) {
             s_slot = 0;
             s_phase ^= 1u;
@@ -825,13 +870,10 @@ __global__ void __launch_bounds__(kThreads, TWO ? 2 : 1)
 __global__ void __launch_bounds__(256) split_rows_kernel(
     const uint16_t* __restrict__ src, const int32_t* __restrict__ gather, int k, int K,
     const Tile* __restrict__ tiles, const int* __restrict__ n_tiles, int NT, int64_t padded_rows,
-    uint8_t* __restrict__ pieces, uint32_t* __restrict__ words, int* __restrict__ work,
-    int* __restrict__ done, int n_done) {
-  // the work counter and the per-tile counts of the GEMM launch that follows
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
-    for (int j = threadIdx.x; j < n_done; j += blockDim.x) done[j] = 0;
-    if (threadIdx.x == 0) *work = 0;
-  }
+    uint8_t* __restrict__ pieces, uint32_t* __restrict__ words) {
+  // the GEMM launch that follows may start; it waits for this kernel before
+  // it reads the pieces or their words
+  allow_dependents();
   const int nstg = (K + BKS - 1) / BKS;
   const int st = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -1041,7 +1083,9 @@ moe_status launch_mlp(const MxPlan& P, const MlpMaps& maps, const MlpArgs& a, in
   // shared memory that no second CTA shares the SM
   const int smem_launch =
       TWO || smem > kMaxSmemPerCta / 2 + 1024 ? smem : kMaxSmemPerCta / 2 + 1024;
-  return launch(grouped_mx_mlp<NT, TWO>, dim3(grid), dim3(kThreads), smem_launch, stream, maps, a);
+  // launched early: it starts while the split kernel before it finishes
+  return launch_ex(grouped_mx_mlp<NT, TWO>, dim3(grid), dim3(kThreads), smem_launch, stream,
+                   true, maps, a);
 }
 
 moe_status launch_nt(const MxPlan& P, const MlpMaps& maps, const MlpArgs& a, int max_items,
@@ -1112,6 +1156,8 @@ moe_status mx_plan(MlpPlan* p, void* ws) {
   P.words_h = reinterpret_cast<uint32_t*>(base + W.words_h);
   P.work = reinterpret_cast<int*>(base + W.sched);
   P.done = P.work + 1;
+  p->sched = P.work;
+  p->n_sched = 1 + static_cast<int>(W.max_tiles);
   const int D = sh.d_model, F = sh.d_ff, E = sh.E;
   if (!make_weight_maps(&P.m_gu, &P.m_gu_t, &P.m_gu2, p->wgu_q, E, 2 * F, D, true) ||
       !make_weight_maps(&P.m_dn, &P.m_dn_t, &P.m_dn2, p->wdn_q, E, D, F, false) ||
@@ -1129,7 +1175,7 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
   const int NT = P.NT, D = sh.d_model, F = sh.d_ff, E = sh.E;
   moe_status st;
   if (!in.tiles_ready &&
-      (st = plan_tiles_launch(in.offsets, E, NT, p.tiles, p.n_tiles, stream)) != MOE_OK)
+      (st = plan_tiles_launch(in.offsets, E, NT, p.tiles, p.n_tiles, p.sched, p.n_sched, stream)) != MOE_OK)
     return st;
   // the input rows, split into pieces (straight from x inside the layer)
   {
@@ -1141,8 +1187,7 @@ moe_status mx_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
                 from_x ? in.x : p.x_perm,
                 from_x ? in.sorted_slot : static_cast<const int32_t*>(nullptr), from_x ? in.k : 1,
                 D, static_cast<const Tile*>(p.tiles), static_cast<const int*>(p.n_tiles), NT,
-                P.padded_rows, P.pieces_x, P.words_x, P.work, P.done,
-                static_cast<int>(P.max_tiles));
+                P.padded_rows, P.pieces_x, P.words_x);
     if (st != MOE_OK) return st;
   }
   const int max_tiles = static_cast<int>(P.max_tiles);

@@ -644,7 +644,7 @@ moe_status bf_enqueue(const MlpPlan& p, const MlpInput& in, int32_t* status, int
   const int max_tiles = static_cast<int>(P.max_tiles);
   moe_status st;
   if (!in.tiles_ready &&
-      (st = plan_tiles_launch(in.offsets, E, NT, p.tiles, p.n_tiles, stream)) != MOE_OK)
+      (st = plan_tiles_launch(in.offsets, E, NT, p.tiles, p.n_tiles, p.sched, p.n_sched, stream)) != MOE_OK)
     return st;
   st = launch_nt<true>(NT, P.m_gu, P.m_x, p.wgu_s, p.tiles, p.n_tiles, F / 64, max_tiles, 2 * F,
                        D, F, p.h, status, fail_cta, stream);

@@ -388,7 +388,7 @@ moe_status unquantised_mlp(const uint16_t* x_perm, const int32_t* offsets, const
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  moe_status st = plan_tiles_launch(offsets, E, NT, tiles, n_tiles, stream);
+  moe_status st = plan_tiles_launch(offsets, E, NT, tiles, n_tiles, nullptr, 0, stream);
   if (st != MOE_OK) return st;
   const int max_tiles = static_cast<int>(W.max_tiles);
   launch_nt<true>(NT, m_gu, m_x, tiles, n_tiles, F / 64, max_tiles, 2 * F, D, F, h, status, stream);

@@ -15,9 +15,11 @@ namespace {
 // experts ascending; one CTA of 256 threads (E <= 256).
 __global__ void __launch_bounds__(256) plan_tiles_kernel(const int32_t* __restrict__ offsets, int E,
                                                          int NT, Tile* __restrict__ tiles,
-                                                         int* __restrict__ n_tiles) {
+                                                         int* __restrict__ n_tiles,
+                                                         int* __restrict__ sched, int n_sched) {
   __shared__ int base[257];
   const int e = threadIdx.x;
+  for (int i = e; i < n_sched; i += blockDim.x) sched[i] = 0;
   int cnt = 0;
   if (e < E) {
     const int c = offsets[e + 1] - offsets[e];
@@ -61,9 +63,9 @@ EncodeTiledFn encode_tiled_fn() {
 }
 
 moe_status plan_tiles_launch(const int32_t* offsets, int E, int NT, Tile* tiles, int* n_tiles,
-                             cudaStream_t stream) {
+                             int* sched, int n_sched, cudaStream_t stream) {
   return launch(plan_tiles_kernel, dim3(1), dim3(256), 0, stream, offsets, E, NT, tiles,
-                n_tiles);
+                n_tiles, sched, n_sched);
 }
 
 // Decode-sized shapes (few routed rows per expert) stream the weights once
@@ -98,6 +100,8 @@ moe_status expert_mlp_plan(const moe_shape& sh, int path, const uint16_t* x_perm
   plan->wdn_s = wdn_s;
   plan->h = h;
   plan->y_perm = y_perm;
+  plan->sched = nullptr;
+  plan->n_sched = 0;
   if (plan->path == kPathBlockScaled) return mx_plan(plan, ws);
   if (!h) return MOE_ERR_INVALID_ARG;
   return bf_plan(plan, ws);

@@ -72,6 +72,10 @@ struct MlpPlan {
   uint16_t *h, *y_perm;
   Tile* tiles;
   int* n_tiles;
+  // counters the GEMM launch needs zeroed beforehand (null when none): the
+  // kernel that writes the tile list zeroes them
+  int* sched;
+  int n_sched;
   MxPlan mx;
   BfPlan bf;
 };
@@ -114,8 +118,9 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 EncodeTiledFn encode_tiled_fn();
 
 // Tile list of the grouped GEMMs on one CTA: expert e contributes
-// ceil(count_e / NT) tiles of up to NT rows, experts ascending.
+// ceil(count_e / NT) tiles of up to NT rows, experts ascending; the same CTA
+// zeroes sched[0, n_sched).
 moe_status plan_tiles_launch(const int32_t* offsets, int E, int NT, Tile* tiles, int* n_tiles,
-                             cudaStream_t stream);
+                             int* sched, int n_sched, cudaStream_t stream);
 
 }  // namespace moe

@@ -33,12 +33,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     permute_kernel(const int32_t* __restrict__ idx, int64_t S, int E, int32_t* __restrict__ counts,
                    int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_slot,
                    int32_t* __restrict__ slot_pos, int NT, Tile* __restrict__ tiles,
-                   int* __restrict__ n_tiles) {
+                   int* __restrict__ n_tiles, int* __restrict__ sched, int n_sched) {
   __shared__ int32_t cnt[kWarps][kMaxE];  // per (warp, expert) count, then running position
   __shared__ int32_t off[kMaxE + 1];
   __shared__ int32_t tbase[kMaxE + 1];    // first tile of each expert (tile list only)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&cnt[0][0])[i] = 0;
+  // the GEMM launch's counters (see MlpPlan::sched)
+  for (int i = threadIdx.x; i < n_sched; i += kThreads) sched[i] = 0;
   __syncthreads();
   const int64_t chunk = (S + kWarps - 1) / kWarps;
   const int64_t lo = S < warp * chunk ? S : warp * chunk;
@@ -158,10 +160,11 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 moe_status permute_launch(const int32_t* idx, const uint16_t* x, const moe_shape& sh,
                           int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
                           int32_t* slot_pos, uint16_t* x_perm, int NT, Tile* tiles,
-                          int* n_tiles, cudaStream_t stream) {
+                          int* n_tiles, int* sched, int n_sched, cudaStream_t stream) {
   const int64_t S = static_cast<int64_t>(sh.T) * sh.k;
   moe_status st = launch(permute_kernel, dim3(1), dim3(kThreads), 0, stream, idx, S,
-                         sh.E, counts, offsets, sorted_slot, slot_pos, NT, tiles, n_tiles);
+                         sh.E, counts, offsets, sorted_slot, slot_pos, NT, tiles, n_tiles,
+                         sched, n_sched);
   if (st != MOE_OK || S == 0 || x_perm == nullptr) return st;
   const int vec = sh.d_model / 8;
   int64_t want = (S * 32 + 255) / 256;
@@ -192,5 +195,5 @@ extern "C" moe_status moe_permute(const int32_t* topk_idx, const uint16_t* x, mo
   moe_status st = check_device();
   if (st != MOE_OK) return st;
   return permute_launch(topk_idx, x, shape, counts, offsets, sorted_slot, slot_pos, x_perm, 0,
-                        nullptr, nullptr, static_cast<cudaStream_t>(stream));
+                        nullptr, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
 }
