@@ -80,16 +80,16 @@ LAUNCH_NOTE = ("step = one replay of a CUDA graph holding one moe_layer_forward 
 
 # dram bytes (read + write) of one moe_expert_mlp call per workload, from ncu
 # captures of the GEMM kernels of the source file named beside them, reported
-# only while that file's code (comments and whitespace aside) still hashes to
-# the value recorded with them
+# only while that file's device code (comments and whitespace aside) still
+# hashes to the value recorded with them
 TRAFFIC: dict[str, tuple[int, str, str]] = {
     # gate/up + down GEMM dram__bytes_read.sum + dram__bytes_write.sum, one
     # launch each, from `ncu --set full` captures of the layer-only benchmark
     "120b_skewed_prefill": (615571200 + 381615104 + 496563968 + 374050048,
-                            "expert_mlp_bf16.cu", "b96e9f861b69c97f"),
+                            "expert_mlp_bf16.cu", "0649cf90e608fef6"),
     # the one launch of both GEMMs
-    "120b_decode": (1609689856 + 11472896, "expert_mlp.cu", "677cfa72aae5d735"),
-    "20b_decode": (429354496 + 5372928, "expert_mlp.cu", "677cfa72aae5d735"),
+    "120b_decode": (1609584640 + 8515584, "expert_mlp.cu", "aa5f9d9df0a4dab7"),
+    "20b_decode": (429360128 + 5184000, "expert_mlp.cu", "aa5f9d9df0a4dab7"),
 }
 
 
@@ -130,9 +130,19 @@ def code_tokens(src: str) -> str:
     return " ".join(src.split())
 
 
+HOST_CODE_MARK = "// ------------------------------------------------------------ host helpers"
+
+
+def device_code(src: str) -> str:
+    """The part of a kernel source file before its host helpers: the kernels
+    and their device functions, which alone decide the DRAM traffic."""
+    cut = src.find(HOST_CODE_MARK)
+    return src if cut < 0 else src[:cut]
+
+
 def kernel_src_sha(name: str) -> str:
     with open(os.path.join(ROOT, "mxfp4_quantised_mixture_b200", "csrc", name)) as f:
-        return hashlib.sha256(code_tokens(f.read()).encode()).hexdigest()[:16]
+        return hashlib.sha256(code_tokens(device_code(f.read())).encode()).hexdigest()[:16]
 
 
 def gemm_path(wl) -> str:
