@@ -516,7 +516,7 @@ def measure_workload(moe, ctx, wl, weights, layer_only=False) -> dict:
             raise RuntimeError("layer reported device status %d" % st)
 
     # the step as a serving loop runs it: moe_layer_forward captured once into
-    # a CUDA graph (its six kernels, no host work per step), replayed per step
+    # a CUDA graph (its five or six kernels, no host work per step), replayed per step
     graph = captured(torch, layer)
     for _ in range(args.warmup):
         flush.fill_(1)

@@ -269,11 +269,13 @@ MOE_API moe_status moe_expert_mlp(const uint16_t* x_perm, const int32_t* offsets
  *         or BF16_DECODE respectively; first 4 bytes = device status word.
  *   test_timeout_cta  testing support, -1 in normal use.  A value c >= 0
  *         makes the first pipeline wait of the MMA issuer in CTA c of the
- *         first GEMM give up after a short bounded wait on a barrier that
+ *         first GEMM launch (on the block-scaled path, the one launch of
+ *         both GEMMs) give up after a short bounded wait on a barrier that
  *         nothing completes, as a real timeout would: the device status
  *         word becomes MOE_ERR_TIMEOUT, every CTA unwinds after draining
- *         its own copies and MMAs, and the outputs are unspecified.  The
- *         next call runs normally.                                        */
+ *         its own copies and MMAs (a CTA waiting on work that CTA c took
+ *         and left undone gives up after the wait limit, 2 s), and the
+ *         outputs are unspecified.  The next call runs normally.          */
 #define MOE_MLP_PATH_AUTO 0
 #define MOE_MLP_PATH_BLOCK_SCALED 1
 #define MOE_MLP_PATH_BF16_DECODE 2

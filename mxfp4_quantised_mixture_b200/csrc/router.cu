@@ -472,7 +472,7 @@ moe_status router_launch(const uint16_t* x, const uint16_t* w_router, int T, int
                          cudaStream_t stream) {
   if (T == 0) return MOE_OK;
   if (static_cast<int64_t>(T) * E <= kSmallRouterWork) {
-    // a few tokens: one CTA per token on the CUDA cores (a tensor-core tile
+    // a few tokens: one or two CTAs per token on the CUDA cores (a tensor-core tile
     // of 128 tokens would be mostly padding, and its reduction over a
     // cluster costs more than the scores)
     // two CTAs per token while the batch leaves half the SMs idle; each then
