@@ -73,3 +73,42 @@ def test_reference_arm_line_on_rank_zero():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"] == "tiny"
+
+
+def test_traffic_records_follow_the_device_code(tmp_path, monkeypatch):
+    # a captured DRAM figure is reported only while the device code of its
+    # kernel file hashes to the recorded value; host code and comments may
+    # change without voiding it
+    sys.path.insert(0, ROOT)
+    import bench
+
+    kernels = "// kernels\n__global__ void k(int* p) { p[0] = 1; }\n"
+    host = bench.HOST_CODE_MARK + "\nint launch() { return 0; }\n"
+    csrc = tmp_path / "mxfp4_quantised_mixture_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text(kernels + host)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.kernel_src_sha("k.cu")
+    monkeypatch.setattr(bench, "TRAFFIC", {"w": (1234, "k.cu", sha)})
+    assert bench.captured_traffic("w") == 1234
+    # host code and comments changed: still the same kernels
+    (csrc / "k.cu").write_text("// another note\n" + kernels + host + "int more() { return 1; }\n")
+    assert bench.captured_traffic("w") == 1234
+    # a kernel changed: the figure is no longer this code's
+    (csrc / "k.cu").write_text(kernels.replace("p[0] = 1", "p[0] = 2") + host)
+    assert bench.captured_traffic("w") is None
+    assert bench.captured_traffic("unrecorded") is None
+
+
+def test_launch_count_per_gemm_path():
+    # the decode workloads take the block-scaled path (five launches per
+    # layer call), the prefill ones the decode-to-bf16 path (six)
+    sys.path.insert(0, ROOT)
+    import bench
+    import synthetic as syn
+
+    want = {"tiny": "block-scaled", "20b_decode": "block-scaled", "120b_decode": "block-scaled",
+            "20b_prefill": "bf16-decode", "120b_skewed_prefill": "bf16-decode"}
+    for name, path in want.items():
+        assert bench.gemm_path(syn.WORKLOADS[name]) == path, name
+    assert bench.LAUNCHES_PER_LAYER == {"block-scaled": 5, "bf16-decode": 6}
